@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark: forward + backward alpha-entmax attention on B200.
+
+One step = entmax_attn_fwd + entmax_attn_bwd (the whole hot path) over one
+batch of the workload, inputs resident in HBM.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Workloads (seeded synthetic data, see differentiable_sparse_attention_b200/workloads.py):
+  alpha15_4k      B=2 H=16 N=4096 D=64 alpha=1.5 causal, q temperature t in {1, 2, 4}
+                  (the default: the sweep the headline metric is quoted on)
+  sparsemax_16k   B=1 H=16 N=16384 D=128 alpha=2 t=3
+  planted_32k     B=1 H=8 N=32768 D=128 alpha=1.5, 32 planted key blocks per head
+  long_sweep      B=1 H=8 D=128 t=4, alpha in {1.5, 2}, N in {65536, 131072}
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+(batch, head) problems are independent: weak scaling, no collective on the
+data path); the timed region is bracketed by barriers and the time is the
+max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import resource
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_points(name: str):
+    if name == "alpha15_4k":
+        return [W.ALPHA15_4K.with_(temperature=t) for t in W.ALPHA15_4K_TEMPERATURES]
+    if name == "sparsemax_16k":
+        return [W.SPARSEMAX_16K]
+    if name == "planted_32k":
+        return [W.PLANTED_32K]
+    if name == "long_sweep":
+        return [W.long_sweep_point(n, a) for n, a in W.LONG_SWEEP_POINTS]
+    if name.startswith("long_n"):
+        n, a = name[len("long_n"):].split("_a")
+        return [W.long_sweep_point(int(n), float(a))]
+    raise SystemExit(f"unknown workload {name}")
+
+
+def effective_flops(w) -> float:
+    """Dense-equivalent FLOPs of fwd + bwd (FlashAttention convention): forward
+    4 N^2 D per head (2 for causal), backward 2.5x the forward."""
+    per_head = (7.0 if w.causal else 14.0) * w.N * w.N * w.D
+    return per_head * w.B * w.H
+
+
+def block_sparsity(mask: torch.Tensor, n: int, block: int, causal: bool) -> float:
+    """1 - |active blocks| / |visible blocks| (causal: blocks i >= j)."""
+    words = mask.to(torch.int64).cpu().numpy() & 0xFFFFFFFF
+    tb = (n + block - 1) // block
+    active = 0
+    for j in range(tb):
+        active += int(((words[..., j // 32] >> (j % 32)) & 1).sum())
+    per_head = tb * (tb + 1) // 2 if causal else tb * tb
+    total = per_head * mask.shape[0] * mask.shape[1]
+    return 1.0 - active / total
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def run_ours(args, points, rank, world, device):
+    import differentiable_sparse_attention_b200 as dsa
+
+    peaks, peaks_kind = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
+    results = []
+    total_eff = 0.0
+    total_ms = 0.0
+    phase_tot = {n: 0.0 for n in dsa.PHASE_NAMES}
+    counters_acc = {}
+    e2e_ms = 0.0
+    h2d = d2h = 0
+    kernel_launches = 0
+
+    for w in points:
+        x = W.make_inputs(w, device="cpu")
+        dev = {k: v.to(device) for k, v in x.items()}
+        B, H, N, D = w.B, w.H, w.N, w.D
+        ws = dsa.alloc_workspace(B, H, N, D, w.block, w.causal, device)
+        out = torch.empty_like(dev["q"])
+        tau = torch.empty((B, H, N), dtype=torch.float32, device=device)
+        mask = torch.empty((B, H, (N + w.block - 1) // w.block, dsa.mask_words(N, w.block)),
+                           dtype=torch.int32, device=device)
+        dq, dk, dv = (torch.empty_like(dev["q"]) for _ in range(3))
+
+        def step(q, k, v, do):
+            dsa.entmax_attn_fwd(q, k, v, w.alpha, w.causal, w.block, out=out, tau=tau, mask=mask,
+                                workspace=ws)
+            dsa.entmax_attn_bwd(q, k, v, do, tau, mask, w.alpha, w.causal, w.block, dq=dq, dk=dk,
+                                dv=dv, workspace=ws)
+
+        for _ in range(max(3, args.warmup)):
+            step(dev["q"], dev["k"], dev["v"], dev["dout"])
+        torch.cuda.synchronize(device)
+        st = dsa.status(ws)
+        cnt = dsa.counters(ws)
+        sparsity = block_sparsity(mask, N, w.block, w.causal)
+
+        # ---- timed region: device-resident inputs, L2 flushed before each step
+        dsa.profile(True)
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(device)
+        ms_steps = []
+        phases = {n: 0.0 for n in dsa.PHASE_NAMES}
+        with ClockSampler(device.index) as clk:
+            for _ in range(args.steps):
+                flush.zero_()
+                ev0.record()
+                step(dev["q"], dev["k"], dev["v"], dev["dout"])
+                ev1.record()
+                ev1.synchronize()
+                ms_steps.append(ev0.elapsed_time(ev1))
+                for n, v in dsa.profile_read().items():
+                    phases[n] += v
+        torch.cuda.synchronize(device)
+        dsa.profile(False)
+        ms_sum = sum(ms_steps)
+        if world > 1:
+            t = torch.tensor([ms_sum], device=device)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms_sum = float(t.item())
+        ms_step = ms_sum / args.steps
+        eff = effective_flops(w)
+        total_eff += eff * args.steps * world
+        total_ms += ms_sum
+        for n in phases:
+            phase_tot[n] += phases[n]
+        for n, v in cnt.items():
+            counters_acc[n] = counters_acc.get(n, 0) + v
+        # our kernels per step: forward; 4 fp16 copies + 2 tile-mask kernels + row + column
+        kernel_launches += args.steps * (1 + 4 + 2 + 2)
+
+        # ---- end to end through the public API: pinned host buffers in and out
+        e2e = None
+        if not args.no_e2e:
+            host_in = {k: v.pin_memory() for k, v in x.items()}
+            host_out = [torch.empty_like(x["q"]).pin_memory() for _ in range(4)]
+            in_bytes = sum(t.numel() * t.element_size() for t in host_in.values())
+            out_bytes = sum(t.numel() * t.element_size() for t in host_out)
+            torch.cuda.synchronize(device)
+            e_ms = []
+            for _ in range(args.steps):
+                flush.zero_()
+                ev0.record()
+                for kname in ("q", "k", "v", "dout"):
+                    dev[kname].copy_(host_in[kname], non_blocking=True)
+                step(dev["q"], dev["k"], dev["v"], dev["dout"])
+                for hb, db in zip(host_out, (out, dq, dk, dv)):
+                    hb.copy_(db, non_blocking=True)
+                ev1.record()
+                ev1.synchronize()
+                e_ms.append(ev0.elapsed_time(ev1))
+            e_sum = sum(e_ms)
+            if world > 1:
+                t = torch.tensor([e_sum], device=device)
+                torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+                e_sum = float(t.item())
+            e2e_ms += e_sum
+            h2d += in_bytes
+            d2h += out_bytes
+            e2e = e_sum / args.steps
+
+        results.append({
+            "point": w.name, "temperature": w.temperature, "alpha": w.alpha, "N": N,
+            "block": w.block, "block_sparsity": round(sparsity, 4),
+            "ms_per_step": round(ms_step, 4),
+            "eff_tflops": round(eff / (ms_step * 1e-3) / 1e12 * world, 2),
+            "phases_ms": {n: round(v / args.steps, 4) for n, v in phases.items()},
+            "counters": cnt, "status": st, "clocks": clk.summary(),
+            "e2e_ms_per_step": None if e2e is None else round(e2e, 4)})
+        del dev, ws, out, tau, mask, dq, dk, dv
+        torch.cuda.empty_cache()
+
+    value = total_eff / (total_ms * 1e-3) / 1e12
+    n_steps_all = args.steps * len(points)
+
+    # ---- roofline of the dominant kernel (by total event time)
+    dom = max(phase_tot, key=phase_tot.get)
+    dom_ms = phase_tot[dom] / n_steps_all
+    roof = roofline_for(dom, dom_ms, points, results, peaks, peaks_kind, args.steps)
+
+    line = {
+        "metric": "fwd+bwd alpha-entmax attn ms/step & effective TFLOP/s vs block sparsity, 1 B200",
+        "value": round(value, 3),
+        "unit": "effective TFLOP/s (dense-equivalent causal 7*B*H*N^2*D per fwd+bwd step)",
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(total_ms / n_steps_all, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1), see workloads.py)",
+        "config": {"workload": args.workload_desc, "l2": "flushed (256 MB write) before every step",
+                   "points": [p["point"] for p in results], "parallelism": f"replica x{world}"},
+        "sweep": results,
+        "kernels_ms_per_step": {n: round(v / n_steps_all, 4) for n, v in phase_tot.items()},
+        "roofline": roof,
+        "gpu_launches": kernel_launches,
+        "clocks": merge_clocks([r["clocks"] for r in results]),
+    }
+    if not args.no_e2e:
+        line["e2e"] = {"value": round(total_eff / (e2e_ms * 1e-3) / 1e12, 3),
+                       "unit": line["unit"], "h2d_bytes_per_step": h2d // len(points),
+                       "d2h_bytes_per_step": d2h // len(points)}
+    return line
+
+
+def merge_clocks(cl):
+    sm = [c["sm_mhz"] for c in cl if c.get("sm_mhz")]
+    reasons = sorted({r for c in cl for r in c.get("reasons", [])})
+    smax = next((c["sm_max_mhz"] for c in cl if c.get("sm_max_mhz")), None)
+    return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax, "reasons": reasons}
+
+
+def roofline_for(kernel, ms, points, results, peaks, peaks_kind, steps):
+    """Achieved vs peak for the dominant kernel.  Tensor-bound kernels count the
+    MMA FLOPs their tile lists imply (128 x 128 tiles):
+      forward:   (hist + refine tiles) * 2*128*128*D + pv tiles * 4*128*128*D
+      bwd row:   row tiles * (2 passes * 2 + 1) * 2*128*128*D   (S, dP twice; dQ)
+      bwd col:   col tiles * 4 * 2*128*128*D                    (S^T, dP^T, dV, dK)
+    """
+    fl = 0.0
+    for w, r in zip(points, results):
+        c = r["counters"]
+        unit = 2.0 * 128 * 128 * w.D
+        if kernel == "fwd":
+            fl += ((c["fwd_hist_tiles"] + c["fwd_refine_tiles"]) + 2 * c["fwd_pv_tiles"]) * unit
+        elif kernel == "bwd_row":
+            fl += c["bwd_row_tiles"] * 5 * unit
+        elif kernel == "bwd_col":
+            fl += c["bwd_col_tiles"] * 4 * unit
+    fl /= len(points)
+    if fl == 0.0:
+        return {"bound": "hbm", "kernel": kernel, "achieved": None, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": None, "traffic": None,
+                "note": f"peak {peaks_kind}"}
+    achieved = fl / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"bound": "tensor", "kernel": kernel, "achieved": round(achieved, 2),
+            "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+            "ms_per_launch": round(ms, 4),
+            "note": f"executed MMA FLOPs per launch / CUDA-event duration; peak = {peaks_kind} "
+                    "dense bf16 burst (fp16 runs at the same rate)"}
+
+
+# ---------------------------------------------------------------- oracle legs
+def oracle_sample(w, n_rows: int):
+    """Time the float64 oracle on n_rows query rows, spread evenly over
+    (batch 0, head 0) of workload w: forward for those rows, then their
+    backward (dQ rows and their dK/dV contributions) reusing the forward's tau.
+    Returns (effective FLOP of the sample, wall seconds, cores used = CPU
+    seconds / wall seconds).  A causal row sees on average N/2 keys, so the
+    sample's dense-equivalent work is the head's 7 N^2 D scaled by n_rows / N."""
+    import oracle as O
+
+    x = W.make_inputs(w.with_(B=1, H=1), device="cpu")
+    q, k, v, do = (W.head_slice(x[n], 0, 0) for n in ("q", "k", "v", "dout"))
+    n_rows = min(n_rows, w.N)
+    rows = np.unique(np.linspace(0, w.N - 1, n_rows).round().astype(np.int64))
+    r0 = resource.getrusage(resource.RUSAGE_SELF)
+    t0 = time.perf_counter()
+    f = O.attention_forward(q, k, v, w.alpha, w.causal, w.block, rows=rows)
+    O.attention_backward(q, k, v, do, w.alpha, w.causal, rows=rows, tau=f["tau"])
+    wall = time.perf_counter() - t0
+    r1 = resource.getrusage(resource.RUSAGE_SELF)
+    cpu = (r1.ru_utime - r0.ru_utime) + (r1.ru_stime - r0.ru_stime)
+    eff = effective_flops(w.with_(B=1, H=1)) * rows.size / w.N
+    return eff, wall, max(1, round(cpu / max(wall, 1e-9))), rows.size
+
+
+def cpu_baseline(points):
+    w = points[0]
+    eff, wall, cores, nr = oracle_sample(w, 2048)
+    return {"value": round(eff / wall / 1e12, 8), "unit": "effective TFLOP/s", "cores": cores,
+            "kind": "oracle", "sample": f"{w.name} t={w.temperature}: {nr} of {w.N} query rows "
+            f"(evenly spread) of batch 0 head 0 (1 of {w.B * w.H} heads), fwd+bwd in float64 "
+            f"NumPy, {wall:.1f} s wall"}
+
+
+def run_reference(args, points, rank, world):
+    """The oracle as it stands, timed on the host cores: every step is a bounded
+    sample (256 evenly spread query rows of batch 0 head 0) of one sweep point,
+    cycling through the points."""
+    if rank != 0:
+        return None
+    total_eff = 0.0
+    total_s = 0.0
+    cores = 1
+    samples = []
+    for i in range(args.steps):
+        w = points[i % len(points)]
+        eff, wall, cores, nr = oracle_sample(w, 256)
+        total_eff += eff
+        total_s += wall
+        samples.append(f"{w.name} t={w.temperature} ({nr} rows)")
+    value = total_eff / total_s / 1e12
+    return {
+        "impl": "reference",
+        "metric": "fwd+bwd alpha-entmax attn ms/step & effective TFLOP/s vs block sparsity, 1 B200",
+        "value": round(value, 8),
+        "unit": "effective TFLOP/s (dense-equivalent causal 7*B*H*N^2*D per fwd+bwd step)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_s * 1e3 / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload_desc,
+                   "sample": "each step = 256 evenly spread query rows of batch 0 head 0 of one "
+                             "sweep point, fwd+bwd through the float64 oracle on host cores"},
+        "cpu_baseline": {"value": round(value, 8), "unit": "effective TFLOP/s", "cores": cores,
+                         "kind": "oracle", "sample": "; ".join(samples)},
+        "e2e": {"value": round(value, 8), "unit": "effective TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="alpha15_4k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    points = workload_points(args.workload)
+    args.workload_desc = (f"{args.workload}: " + ", ".join(
+        f"B={p.B} H={p.H} N={p.N} D={p.D} alpha={p.alpha} t={p.temperature}"
+        + (f" planted={p.planted_blocks}" if p.planted_blocks else "") for p in points)
+        + f"; causal, block {points[0].block}, bf16")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, points, rank, world)
+        if line is not None:
+            print(json.dumps(line))
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=device,
+                                             timeout=datetime.timedelta(seconds=120))
+    line = run_ours(args, points, rank, world, device)
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(points)
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

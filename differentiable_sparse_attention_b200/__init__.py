@@ -1,0 +1,226 @@
+"""alpha-entmax attention (forward + backward) for NVIDIA B200, sm_100a.
+
+A thin ctypes binding of ``libentmax_attn.so``, whose C ABI is declared in
+``include/entmax_attn.h``.  This module only marshals arguments: every step of
+the computation runs in the library's CUDA kernels, and there is no fallback
+of any kind -- if the library is missing, the calls raise.
+PyTorch provides device memory and the current CUDA stream.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libentmax_attn.so")
+
+OK = 0
+E_NULL, E_ALIGN, E_SHAPE, E_UNSUPPORTED, E_ALPHA, E_WORKSPACE, E_CUDA, E_MAXITER = (
+    -1, -2, -3, -4, -5, -6, -7, -8)
+ST_NOT_CONVERGED, ST_TIMEOUT, ST_RANGE = 1, 2, 4
+DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
+EXPORTED = ("entmax_attn_mask_words", "entmax_attn_workspace_size", "entmax_attn_fwd",
+            "entmax_attn_bwd", "entmax_attn_status", "entmax_attn_counters",
+            "entmax_attn_profile", "entmax_attn_profile_read", "entmax_attn_error_string")
+COUNTER_NAMES = ("fwd_hist_tiles", "fwd_refine_tiles", "fwd_pv_tiles", "fwd_refine_passes",
+                 "bwd_row_tiles", "bwd_col_tiles")
+PHASE_NAMES = ("fwd", "bwd_fp16_copies", "bwd_tile_masks", "bwd_row", "bwd_col")
+
+_lib_handle = None
+
+
+class EntmaxError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what} failed with {code}: {error_string(code)}")
+
+
+def _lib():
+    """Load the shared library (once).  Raises if it has not been built."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing; build it with "
+            "`python -m differentiable_sparse_attention_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    c_int, c_float, c_size, vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+    lib.entmax_attn_mask_words.argtypes = [c_int, c_int]
+    lib.entmax_attn_mask_words.restype = c_int
+    lib.entmax_attn_workspace_size.argtypes = [c_int] * 6
+    lib.entmax_attn_workspace_size.restype = c_size
+    lib.entmax_attn_fwd.argtypes = ([vp, vp, vp] + [c_int] * 5 + [c_float, c_int, c_int, c_int]
+                                    + [vp] * 5 + [c_size, vp])
+    lib.entmax_attn_fwd.restype = c_int
+    lib.entmax_attn_bwd.argtypes = ([vp] * 6 + [c_int] * 5 + [c_float, c_int, c_int]
+                                    + [vp] * 4 + [c_size, vp])
+    lib.entmax_attn_bwd.restype = c_int
+    lib.entmax_attn_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.entmax_attn_status.restype = c_int
+    lib.entmax_attn_counters.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_ulonglong), c_int]
+    lib.entmax_attn_counters.restype = c_int
+    lib.entmax_attn_profile.argtypes = [c_int]
+    lib.entmax_attn_profile.restype = c_int
+    lib.entmax_attn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), c_int]
+    lib.entmax_attn_profile_read.restype = c_int
+    lib.entmax_attn_error_string.argtypes = [c_int]
+    lib.entmax_attn_error_string.restype = ctypes.c_char_p
+    _lib_handle = lib
+    return lib
+
+
+def error_string(code: int) -> str:
+    return _lib().entmax_attn_error_string(int(code)).decode()
+
+
+def mask_words(n: int, block: int) -> int:
+    w = _lib().entmax_attn_mask_words(int(n), int(block))
+    if w < 0:
+        raise EntmaxError(w, "entmax_attn_mask_words")
+    return w
+
+
+def workspace_size(B: int, H: int, N: int, D: int, block: int = 128, causal: bool = True) -> int:
+    return int(_lib().entmax_attn_workspace_size(B, H, N, D, block, int(bool(causal))))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream, device):
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_qkv(*ts):
+    ref = ts[0]
+    for t in ts:
+        if t.dim() != 4 or t.shape != ref.shape or t.dtype != ref.dtype or not t.is_contiguous():
+            raise ValueError("q, k, v (, dout) must be contiguous [B, H, N, D] tensors of one dtype")
+        if t.device != ref.device or t.device.type != "cuda":
+            raise ValueError("tensors must live on one CUDA device")
+    if ref.dtype not in DTYPE_CODES:
+        raise ValueError(f"unsupported dtype {ref.dtype}")
+
+
+class FwdResult(NamedTuple):
+    out: torch.Tensor
+    tau: torch.Tensor
+    mask: torch.Tensor
+    workspace: torch.Tensor
+    tau_trace: Optional[torch.Tensor]
+
+
+def alloc_workspace(B, H, N, D, block=128, causal=True, device="cuda"):
+    return torch.empty(workspace_size(B, H, N, D, block, causal), dtype=torch.uint8, device=device)
+
+
+def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = True, block: int = 128,
+                    max_iter: int = 4, *, out=None, tau=None, mask=None, workspace=None,
+                    trace: bool = False, stream=None) -> FwdResult:
+    """alpha-entmax attention forward through ``entmax_attn_fwd``."""
+    _check_qkv(q, k, v)
+    B, H, N, D = q.shape
+    dev = q.device
+    out = torch.empty_like(q) if out is None else out
+    tau = torch.empty((B, H, N), dtype=torch.float32, device=dev) if tau is None else tau
+    mrows = (N + block - 1) // block
+    if mask is None:
+        mask = torch.empty((B, H, mrows, mask_words(N, block)), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, D, block, causal, dev)
+    trace_t = (torch.empty((max_iter + 1, B, H, N), dtype=torch.float32, device=dev)
+               if trace else None)
+    rc = _lib().entmax_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), B, H, N, D, DTYPE_CODES[q.dtype], float(alpha),
+        int(bool(causal)), int(block), int(max_iter), _ptr(out), _ptr(tau), _ptr(mask),
+        _ptr(trace_t), _ptr(workspace), workspace.numel(), _stream_ptr(stream, dev))
+    if rc != OK:
+        raise EntmaxError(rc, "entmax_attn_fwd")
+    return FwdResult(out, tau, mask, workspace, trace_t)
+
+
+def entmax_attn_bwd(q, k, v, dout, tau, mask, alpha: float = 1.5, causal: bool = True,
+                    block: int = 128, *, dq=None, dk=None, dv=None, workspace=None,
+                    stream=None):
+    """alpha-entmax attention backward through ``entmax_attn_bwd``; returns (dq, dk, dv)."""
+    _check_qkv(q, k, v, dout)
+    B, H, N, D = q.shape
+    dev = q.device
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, D, block, causal, dev)
+    rc = _lib().entmax_attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(tau), _ptr(mask), B, H, N, D,
+        DTYPE_CODES[q.dtype], float(alpha), int(bool(causal)), int(block), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(workspace), workspace.numel(), _stream_ptr(stream, dev))
+    if rc != OK:
+        raise EntmaxError(rc, "entmax_attn_bwd")
+    return dq, dk, dv
+
+
+def status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream and return the device status bits (ST_*)."""
+    word = ctypes.c_uint32(0)
+    rc = _lib().entmax_attn_status(_ptr(workspace), _stream_ptr(stream, workspace.device),
+                                   ctypes.byref(word))
+    if rc != OK:
+        raise EntmaxError(rc, "entmax_attn_status")
+    return int(word.value)
+
+
+def counters(workspace: torch.Tensor, stream=None) -> dict:
+    """Synchronise the stream and return the work counters (COUNTER_NAMES)."""
+    arr = (ctypes.c_ulonglong * len(COUNTER_NAMES))()
+    rc = _lib().entmax_attn_counters(_ptr(workspace), _stream_ptr(stream, workspace.device), arr,
+                                     len(COUNTER_NAMES))
+    if rc != OK:
+        raise EntmaxError(rc, "entmax_attn_counters")
+    return dict(zip(COUNTER_NAMES, (int(x) for x in arr)))
+
+
+def profile(enable: bool) -> None:
+    """Turn per-kernel CUDA-event recording on or off for this thread."""
+    rc = _lib().entmax_attn_profile(int(bool(enable)))
+    if rc != OK:
+        raise EntmaxError(rc, "entmax_attn_profile")
+
+
+def profile_read() -> dict:
+    """Per-kernel milliseconds of this thread's last recorded fwd / bwd calls."""
+    arr = (ctypes.c_float * len(PHASE_NAMES))()
+    rc = _lib().entmax_attn_profile_read(arr, len(PHASE_NAMES))
+    if rc != OK:
+        raise EntmaxError(rc, "entmax_attn_profile_read")
+    return dict(zip(PHASE_NAMES, (float(x) for x in arr)))
+
+
+class EntmaxAttention(torch.autograd.Function):
+    """autograd wrapper: O = entmax_attention(q, k, v); backward through the library."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, alpha=1.5, causal=True, block=128, max_iter=4):
+        r = entmax_attn_fwd(q, k, v, alpha, causal, block, max_iter)
+        ctx.save_for_backward(q, k, v, r.tau, r.mask, r.workspace)
+        ctx.cfg = (alpha, causal, block)
+        return r.out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, tau, mask, ws = ctx.saved_tensors
+        alpha, causal, block = ctx.cfg
+        dq, dk, dv = entmax_attn_bwd(q, k, v, dout.contiguous(), tau, mask, alpha, causal, block,
+                                     workspace=ws)
+        return dq, dk, dv, None, None, None, None
+
+
+def entmax_attention(q, k, v, alpha=1.5, causal=True, block=128, max_iter=4):
+    return EntmaxAttention.apply(q, k, v, alpha, causal, block, max_iter)

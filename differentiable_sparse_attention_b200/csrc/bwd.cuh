@@ -1,0 +1,756 @@
+// Backward alpha-entmax attention kernels for sm_100a.
+//
+// The backward visits only the blocks the forward's bit-packed mask marks
+// active (AdaSplash-2 zh §2.3, it §2C, ja §2.3: zero blocks are skipped in the
+// backward too, and local accumulators replace atomics).  With
+// t = [s - tau]_+, p = t^(1/(alpha-1)) and g = p^(2-alpha) (g = t at alpha = 1.5,
+// g = 1[t > 0] at alpha = 2):
+//     dP = dO V^T,   delta_r = sum_c g dP / sum_c g,   dZ = g (dP - delta)
+//     dQ = dZ K / sqrt(D),   dK = dZ^T Q / sqrt(D),   dV = P^T dO
+//
+//   tile_mask_kernel / tile_mask_t_kernel  block mask -> 128x128 tile mask and its
+//                                          transpose (workspace)
+//   entmax_bwd_row_kernel   one CTA per 128-row query tile: pass A computes
+//                           delta over the active key tiles, pass B dQ.
+//   entmax_bwd_col_kernel   one CTA per 128-key tile: dK and dV over the active
+//                           query tiles, accumulated in TMEM (no atomics).
+#pragma once
+
+#include "common.cuh"
+
+namespace entmax {
+
+// ----------------------------------------------------------------- masks
+// tm[bh][i][w]: bit (j % 32) of word w = j / 32 is set iff any block of the
+// (block)-granularity mask inside 128x128 tile (i, j) is set.
+__global__ void tile_mask_kernel(const uint32_t* __restrict__ mask, uint32_t* __restrict__ tm,
+                                 int BH, int T, int block, int mask_rows, int mask_words) {
+  const int wt = (T + 31) / 32;
+  const long long total = static_cast<long long>(BH) * T * wt;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int w = static_cast<int>(idx % wt);
+    const int i = static_cast<int>((idx / wt) % T);
+    const int bh = static_cast<int>(idx / (static_cast<long long>(wt) * T));
+    const uint32_t* mrow = mask + static_cast<size_t>(bh) * mask_rows * mask_words;
+    uint32_t out = 0u;
+    if (block == kTile) {
+      out = mrow[static_cast<size_t>(i) * mask_words + w];
+    } else {  // 64: rows 2i, 2i+1 and key blocks 2j, 2j+1
+      for (int a = 0; a < 2; ++a) {
+        const int r = 2 * i + a;
+        if (r >= mask_rows) continue;
+        for (int bit = 0; bit < 32; ++bit) {
+          const int j = w * 32 + bit;
+          if (j >= T) break;
+          const int kb = 2 * j;
+          const uint32_t two = (mrow[static_cast<size_t>(r) * mask_words + (kb >> 5)] >> (kb & 31)) & 3u;
+          if (two) out |= 1u << bit;
+        }
+      }
+    }
+    tm[idx] = out;
+  }
+}
+
+// tmt[bh][j][w]: bit (i % 32) of word i / 32 = tm[bh][i] bit j.
+__global__ void tile_mask_t_kernel(const uint32_t* __restrict__ tm, uint32_t* __restrict__ tmt,
+                                   int BH, int T) {
+  const int wt = (T + 31) / 32;
+  const long long total = static_cast<long long>(BH) * T * wt;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int w = static_cast<int>(idx % wt);
+    const int j = static_cast<int>((idx / wt) % T);
+    const int bh = static_cast<int>(idx / (static_cast<long long>(wt) * T));
+    const uint32_t* base = tm + static_cast<size_t>(bh) * T * wt;
+    uint32_t out = 0u;
+    for (int bit = 0; bit < 32; ++bit) {
+      const int i = w * 32 + bit;
+      if (i >= T) break;
+      out |= ((base[static_cast<size_t>(i) * wt + (j >> 5)] >> (j & 31)) & 1u) << bit;
+    }
+    tmt[idx] = out;
+  }
+}
+
+// bf16 -> fp16 copy of the backward's inputs (exact for |x| in [2^-14, 65504]:
+// 8 significant bits fit in fp16's 11).  The backward runs its MMAs in fp16 so
+// that the rounded operands built on chip (P and dS) keep 11 significant bits
+// instead of bf16's 8; |x| > 65504 raises ST_RANGE.
+__global__ void to_fp16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
+                               size_t n8, uint32_t* status) {
+  bool bad = false;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 in = reinterpret_cast<const uint4*>(src)[i];
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
+      const float2 f = __bfloat1622float2(b);
+      bad |= !(fabsf(f.x) <= 65504.0f) || !(fabsf(f.y) <= 65504.0f);
+      const __half2 h = __floats2half2_rn(f.x, f.y);
+      o[e] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    reinterpret_cast<uint4*>(dst)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (bad) atomicOr(status, ST_RANGE);
+}
+
+struct BwdParams {
+  int BH, N, T, wt;          // T = 128-tiles per side, wt = words per tile-mask row
+  int causal;
+  float c;                   // (alpha - 1) / sqrt(D)
+  float inv_sqrt_d;
+  const float* tau;          // [BH][N]
+  const uint32_t* tm;        // tile mask rows (row kernel) or transposed rows (column kernel)
+  float* delta;              // workspace [BH][N]
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  uint32_t* status;
+  unsigned long long* counters;
+};
+
+// Loads the tile list of row `r` of a [BH][T][wt] bit matrix into smem
+// (executed by one warp; find-first-set / popcount traversal).
+__device__ __forceinline__ int load_tile_list(const uint32_t* rowbits, int wt, uint16_t* tiles) {
+  const int lane = threadIdx.x & 31;
+  int total = 0;
+  for (int base = 0; base < wt; base += 32) {
+    const int w = base + lane;
+    uint32_t word = (w < wt) ? rowbits[w] : 0u;
+    const int cnt = __popc(word);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int pos = total + incl - cnt;
+    while (word) {
+      const int b = __ffs(word) - 1;
+      tiles[pos++] = static_cast<uint16_t>(w * 32 + b);
+      word &= word - 1u;
+    }
+    total += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return total;
+}
+
+// ============================================================ row kernel (delta, dQ)
+template <int D, int NSK, int NSV>
+struct BwdRowSmem {
+  __half q[kTile * D];
+  __half dout[kTile * D];
+  __half k[NSK][kTile * D];
+  __half v[NSV][kTile * D];
+  __half ds[kTile * kTile];   // dS tile, K-major (K = keys)
+  uint64_t qdo_full;
+  uint64_t k_full[NSK], k_empty[NSK];
+  uint64_t v_full[NSV], v_empty[NSV];
+  uint64_t s_full, s_empty, ds_full, ds_empty, dq_full, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int ntiles;
+  uint16_t tiles[kMaxTiles];
+};
+
+template <int D, int NSK, int NSV>
+constexpr size_t bwd_row_smem_bytes() {
+  return sizeof(BwdRowSmem<D, NSK, NSV>) + 1024;
+}
+
+template <int D, int NSK, int NSV, bool ALPHA2>
+__global__ void __launch_bounds__(kThreads, 1)
+    entmax_bwd_row_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_do, const BwdParams P) {
+  static_assert(NSK >= 2, "pass B keeps K(t-1) while S(t) is issued");
+  extern __shared__ uint8_t smem_raw[];
+  auto& sm = *reinterpret_cast<BwdRowSmem<D, NSK, NSV>*>(align1024(smem_raw));
+  constexpr int kSlabs = D / 64;
+  constexpr uint32_t kTileBytes = kTile * D * 2;
+  constexpr uint32_t kIdescS = make_idesc(kTile, kTile, 0, 0, 0, 0);  // [128 x D] x [128 x D]^T, f16
+  constexpr uint32_t kIdescDQ = make_idesc(kTile, D, 0, 0, 0, 1);     // dS (K-major) x K (MN-major)
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int i = P.T - 1 - static_cast<int>(blockIdx.x) / P.BH;
+  const int bh = static_cast<int>(blockIdx.x) % P.BH;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.qdo_full, 1);
+    for (int s = 0; s < NSK; ++s) { mbar_init(&sm.k_full[s], 1); mbar_init(&sm.k_empty[s], 1); }
+    for (int s = 0; s < NSV; ++s) { mbar_init(&sm.v_full[s], 1); mbar_init(&sm.v_empty[s], 1); }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.s_empty, 4);
+    mbar_init(&sm.ds_full, 4);
+    mbar_init(&sm.ds_empty, 1);
+    mbar_init(&sm.dq_full, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    const int n = load_tile_list(P.tm + (static_cast<size_t>(bh) * P.T + i) * P.wt, P.wt, sm.tiles);
+    if (lane == 0) {
+      sm.ntiles = n;
+      atomicAdd(&P.counters[CNT_ROW_TILES], static_cast<unsigned long long>(n));
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int n = sm.ntiles;
+  volatile int* abort_flag = &sm.abort_flag;
+  uint32_t kc = 0, vc = 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      mbar_expect_tx(&sm.qdo_full, 2 * kTileBytes);
+      for (int s = 0; s < kSlabs; ++s) {
+        tma_load_3d(sm.q + s * kTile * 64, &tm_q, &sm.qdo_full, s * 64, i * kTile, bh);
+        tma_load_3d(sm.dout + s * kTile * 64, &tm_do, &sm.qdo_full, s * 64, i * kTile, bh);
+      }
+      for (int pass = 0; pass < 2 && ok; ++pass) {
+        for (int t = 0; t < n && ok; ++t) {
+          const int j = sm.tiles[t];
+          {
+            const uint32_t slot = kc % NSK, use = kc / NSK;
+            if (use > 0 && !mbar_wait(&sm.k_empty[slot], (use - 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            mbar_expect_tx(&sm.k_full[slot], kTileBytes);
+            for (int s = 0; s < kSlabs; ++s)
+              tma_load_3d(sm.k[slot] + s * kTile * 64, &tm_k, &sm.k_full[slot], s * 64, j * kTile, bh);
+            ++kc;
+          }
+          {
+            const uint32_t slot = vc % NSV, use = vc / NSV;
+            if (use > 0 && !mbar_wait(&sm.v_empty[slot], (use - 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            mbar_expect_tx(&sm.v_full[slot], kTileBytes);
+            for (int s = 0; s < kSlabs; ++s)
+              tma_load_3d(sm.v[slot] + s * kTile * 64, &tm_v, &sm.v_full[slot], s * 64, j * kTile, bh);
+            ++vc;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(&sm.qdo_full, 0, abort_flag, P.status);
+      const uint32_t q_addr = smem_u32(sm.q), do_addr = smem_u32(sm.dout);
+      uint32_t sc = 0, dc = 0;
+      uint32_t kslot_prev = 0;
+      // S = Q K^T and dP = dO V^T of the next tile into TMEM.
+      auto issue_sdp = [&](bool release_k) -> bool {
+        const uint32_t ks = kc % NSK, vs = vc % NSV;
+        if (!mbar_wait(&sm.k_full[ks], (kc / NSK) & 1, abort_flag, P.status)) return false;
+        if (!mbar_wait(&sm.v_full[vs], (vc / NSV) & 1, abort_flag, P.status)) return false;
+        if (sc > 0 && !mbar_wait(&sm.s_empty, (sc - 1) & 1, abort_flag, P.status)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sm.k[ks]), v_addr = smem_u32(sm.v[vs]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+          mma_f16_ss(tmem + kColS, smem_desc_sw128(q_addr + off, 16, 1024),
+                     smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          mma_f16_ss(tmem + kColDP, smem_desc_sw128(do_addr + off, 16, 1024),
+                     smem_desc_sw128(v_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sm.s_full);
+        mma_commit(&sm.v_empty[vs]);
+        if (release_k) mma_commit(&sm.k_empty[ks]);
+        kslot_prev = ks;
+        ++kc;
+        ++vc;
+        ++sc;
+        return true;
+      };
+      // dQ += dS K of the previous tile (K slot kslot).
+      auto issue_dq = [&](uint32_t kslot) -> bool {
+        if (!mbar_wait(&sm.ds_full, dc & 1, abort_flag, P.status)) return false;
+        tc_fence_after();
+        const uint32_t ds_addr = smem_u32(sm.ds), k_addr = smem_u32(sm.k[kslot]);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint32_t a_off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+          mma_f16_ss(tmem + kColDQ, smem_desc_sw128(ds_addr + a_off, 16, 1024),
+                     smem_desc_sw128(k_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescDQ,
+                     (dc > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&sm.ds_empty);
+        mma_commit(&sm.k_empty[kslot]);
+        ++dc;
+        return true;
+      };
+      // pass A: delta
+      for (int t = 0; t < n && ok; ++t) ok = issue_sdp(true);
+      // pass B: dQ, software-pipelined by one tile
+      uint32_t pending = 0;
+      for (int t = 0; t <= n && ok; ++t) {
+        uint32_t this_slot = 0;
+        if (t < n) {
+          ok = issue_sdp(false);
+          this_slot = kslot_prev;
+        }
+        if (ok && t > 0) ok = issue_dq(pending);
+        pending = this_slot;
+      }
+      if (ok) mma_commit(&sm.dq_full);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const int rl = quad * 32 + lane;
+    const int row = i * kTile + rl;
+    const bool row_ok = row < P.N;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float tau_r = row_ok ? P.tau[static_cast<size_t>(bh) * P.N + row] : INFINITY;
+    bool ok = true;
+    uint32_t sc = 0, dc = 0;
+    double gdp = 0.0, gsum = 0.0;
+    float delta = 0.0f;
+    uint8_t* ds_base = reinterpret_cast<uint8_t*>(sm.ds);
+
+    auto valid_col = [&](int col) { return col < P.N && (!P.causal || col <= row); };
+
+    for (int pass = 0; pass < 2 && ok; ++pass) {
+      for (int t = 0; t < n; ++t) {
+        const int j = sm.tiles[t];
+        ok = mbar_wait(&sm.s_full, sc & 1, abort_flag, P.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++sc;
+        tc_fence_after();
+        if (pass == 1 && dc > 0) {
+          ok = mbar_wait(&sm.ds_empty, (dc - 1) & 1, abort_flag, P.status);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+        }
+        const bool msk = (P.causal && j == i) || ((j + 1) * kTile > P.N);
+        float a_gdp = 0.f, a_g = 0.f;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t rs[32], rp[32];
+          tmem_ld32x2(t_lane + kColS + ch * 32, rs, t_lane + kColDP + ch * 32, rp);
+          if (ch == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.s_empty);
+          }
+          float gg[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float tt = fmaf(__uint_as_float(rs[e]), P.c, -tau_r);
+            if (msk && !valid_col(j * kTile + ch * 32 + e)) tt = -1.0f;
+            gg[e] = ALPHA2 ? (tt > 0.f ? 1.f : 0.f) : fmaxf(tt, 0.f);
+          }
+          if (pass == 0) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              a_gdp = fmaf(gg[e], __uint_as_float(rp[e]), a_gdp);
+              a_g += gg[e];
+            }
+          } else {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float d0 = gg[2 * e] * (__uint_as_float(rp[2 * e]) - delta);
+              const float d1 = gg[2 * e + 1] * (__uint_as_float(rp[2 * e + 1]) - delta);
+              const __half2 h2 = __floats2half2_rn(d0, d1);
+              w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd)
+              *reinterpret_cast<uint4*>(ds_base + sw128_chunk_offset(rl, ch * 4 + qd)) =
+                  make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
+          }
+        }
+        if (pass == 0) {
+          gdp += a_gdp;
+          gsum += a_g;
+        } else {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.ds_full);
+          ++dc;
+        }
+      }
+      if (pass == 0) {
+        delta = gsum > 0.0 ? static_cast<float>(gdp / gsum) : 0.0f;
+        if (row_ok) P.delta[static_cast<size_t>(bh) * P.N + row] = delta;
+      }
+    }
+    // dQ epilogue
+    if (ok && n > 0) {
+      ok = mbar_wait(&sm.dq_full, 0, abort_flag, P.status);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    tc_fence_after();
+    __nv_bfloat16* dst_row = P.dq + (static_cast<size_t>(bh) * P.N + row) * D;
+#pragma unroll 1
+    for (int ch = 0; ch < D / 32; ++ch) {
+      uint32_t r[32];
+      if (ok && n > 0) {
+        tmem_ld32(t_lane + kColDQ + ch * 32, r);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = 0u;
+      }
+      if (row_ok) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const __nv_bfloat162 h2 =
+              __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * P.inv_sqrt_d,
+                                    __uint_as_float(r[2 * e + 1]) * P.inv_sqrt_d);
+          w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 32);
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd)
+          dst[qd] = make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (sm.abort_flag) {
+    if (warp == 0 && lane == 0) {
+      mbar_wait(&sm.qdo_full, 0, nullptr, nullptr);
+      for (uint32_t s = 0; s < NSK; ++s)
+        if (kc > s) mbar_wait(&sm.k_full[s], ((kc - 1 - s) / NSK) & 1, nullptr, nullptr);
+      for (uint32_t s = 0; s < NSV; ++s)
+        if (vc > s) mbar_wait(&sm.v_full[s], ((vc - 1 - s) / NSV) & 1, nullptr, nullptr);
+    }
+    if (warp == 1 && lane == 0) {
+      mma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, nullptr, nullptr);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================ column kernel (dK, dV)
+template <int D, int NS>
+struct BwdColSmem {
+  __half k[kTile * D];
+  __half v[kTile * D];
+  __half q[NS][kTile * D];
+  __half dout[NS][kTile * D];
+  __half pt[kTile * kTile];    // P^T tile  [keys][rows], K-major (K = rows)
+  __half dst[kTile * kTile];   // dS^T tile [keys][rows]
+  float tau[NS][kTile];
+  float delta[NS][kTile];
+  uint64_t kv_full;
+  uint64_t q_full[NS], q_empty[NS];
+  uint64_t s_full, s_empty, pt_full, pt_empty, acc_full, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int ntiles;
+  uint16_t tiles[kMaxTiles];
+};
+
+template <int D, int NS>
+constexpr size_t bwd_col_smem_bytes() {
+  return sizeof(BwdColSmem<D, NS>) + 1024;
+}
+
+template <int D, int NS, bool ALPHA2>
+__global__ void __launch_bounds__(kThreads, 1)
+    entmax_bwd_col_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_do, const BwdParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  auto& sm = *reinterpret_cast<BwdColSmem<D, NS>*>(align1024(smem_raw));
+  constexpr int kSlabs = D / 64;
+  constexpr uint32_t kTileBytes = kTile * D * 2;
+  constexpr uint32_t kIdescS = make_idesc(kTile, kTile, 0, 0, 0, 0);   // K Q^T, V dO^T, f16
+  constexpr uint32_t kIdescAcc = make_idesc(kTile, D, 0, 0, 0, 1);    // P^T dO, dS^T Q
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // causal: key tile j is seen by T - j row tiles, so small j first
+  const int j = static_cast<int>(blockIdx.x) / P.BH;
+  const int bh = static_cast<int>(blockIdx.x) % P.BH;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.kv_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sm.q_full[s], 1 + 32);  // TMA expect_tx + 32 lanes staging tau/delta
+      mbar_init(&sm.q_empty[s], 1);
+    }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.s_empty, 4);
+    mbar_init(&sm.pt_full, 4);
+    mbar_init(&sm.pt_empty, 1);
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    const int n = load_tile_list(P.tm + (static_cast<size_t>(bh) * P.T + j) * P.wt, P.wt, sm.tiles);
+    if (lane == 0) {
+      sm.ntiles = n;
+      atomicAdd(&P.counters[CNT_COL_TILES], static_cast<unsigned long long>(n));
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int n = sm.ntiles;
+  volatile int* abort_flag = &sm.abort_flag;
+  uint32_t qc = 0;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    bool ok = true;
+    if (lane == 0) {
+      mbar_expect_tx(&sm.kv_full, 2 * kTileBytes);
+      for (int s = 0; s < kSlabs; ++s) {
+        tma_load_3d(sm.k + s * kTile * 64, &tm_k, &sm.kv_full, s * 64, j * kTile, bh);
+        tma_load_3d(sm.v + s * kTile * 64, &tm_v, &sm.kv_full, s * 64, j * kTile, bh);
+      }
+    }
+    for (int t = 0; t < n && ok; ++t) {
+      const int it = sm.tiles[t];
+      const uint32_t slot = qc % NS, use = qc / NS;
+      if (use > 0) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&sm.q_empty[slot], (use - 1) & 1, abort_flag, P.status);
+        ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+        __syncwarp();
+        if (!ok) break;
+      }
+      if (lane == 0) {
+        mbar_expect_tx(&sm.q_full[slot], 2 * kTileBytes);
+        for (int s = 0; s < kSlabs; ++s) {
+          tma_load_3d(sm.q[slot] + s * kTile * 64, &tm_q, &sm.q_full[slot], s * 64, it * kTile, bh);
+          tma_load_3d(sm.dout[slot] + s * kTile * 64, &tm_do, &sm.q_full[slot], s * 64, it * kTile, bh);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = lane * 4 + e;
+        const int row = it * kTile + r;
+        const size_t g = static_cast<size_t>(bh) * P.N + row;
+        sm.tau[slot][r] = row < P.N ? P.tau[g] : INFINITY;
+        sm.delta[slot][r] = row < P.N ? P.delta[g] : 0.0f;
+      }
+      mbar_arrive(&sm.q_full[slot]);
+      ++qc;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&sm.kv_full, 0, abort_flag, P.status);
+      const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+      uint32_t sc = 0, ac = 0;
+      auto issue_s = [&](uint32_t slot, uint32_t use) -> bool {
+        if (!mbar_wait(&sm.q_full[slot], use & 1, abort_flag, P.status)) return false;
+        if (sc > 0 && !mbar_wait(&sm.s_empty, (sc - 1) & 1, abort_flag, P.status)) return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sm.q[slot]), do_addr = smem_u32(sm.dout[slot]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+          mma_f16_ss(tmem + kColS, smem_desc_sw128(k_addr + off, 16, 1024),
+                     smem_desc_sw128(q_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          mma_f16_ss(tmem + kColDP, smem_desc_sw128(v_addr + off, 16, 1024),
+                     smem_desc_sw128(do_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sm.s_full);
+        ++sc;
+        return true;
+      };
+      auto issue_acc = [&](uint32_t slot) -> bool {
+        if (!mbar_wait(&sm.pt_full, ac & 1, abort_flag, P.status)) return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sm.q[slot]), do_addr = smem_u32(sm.dout[slot]);
+        const uint32_t pt_addr = smem_u32(sm.pt), ds_addr = smem_u32(sm.dst);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint32_t a_off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+          const uint32_t b_off = kk * 16 * 128;
+          const uint32_t acc = (ac > 0 || kk > 0) ? 1u : 0u;
+          mma_f16_ss(tmem + kColDV, smem_desc_sw128(pt_addr + a_off, 16, 1024),
+                     smem_desc_sw128(do_addr + b_off, kSlabBytes, 1024), kIdescAcc, acc);
+          mma_f16_ss(tmem + kColDK, smem_desc_sw128(ds_addr + a_off, 16, 1024),
+                     smem_desc_sw128(q_addr + b_off, kSlabBytes, 1024), kIdescAcc, acc);
+        }
+        mma_commit(&sm.pt_empty);
+        mma_commit(&sm.q_empty[slot]);
+        ++ac;
+        return true;
+      };
+      if (NS >= 2) {
+        for (int t = 0; t <= n && ok; ++t) {
+          if (t < n) ok = issue_s(t % NS, t / NS);
+          if (ok && t > 0) ok = issue_acc((t - 1) % NS);
+        }
+      } else {
+        for (int t = 0; t < n && ok; ++t) {
+          ok = issue_s(0, t);
+          if (ok) ok = issue_acc(0);
+        }
+      }
+      if (ok) mma_commit(&sm.acc_full);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const int kl = quad * 32 + lane;          // key within the tile
+    const int key = j * kTile + kl;
+    const bool key_ok = key < P.N;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    bool ok = true;
+    uint32_t sc = 0, ac = 0;
+    uint8_t* pt_base = reinterpret_cast<uint8_t*>(sm.pt);
+    uint8_t* ds_base = reinterpret_cast<uint8_t*>(sm.dst);
+    for (int t = 0; t < n; ++t) {
+      const int it = sm.tiles[t];
+      const uint32_t slot = t % NS, use = t / NS;
+      ok = mbar_wait(&sm.s_full, sc & 1, abort_flag, P.status) &&
+           mbar_wait(&sm.q_full[slot], use & 1, abort_flag, P.status);
+      if (ok && ac > 0) ok = mbar_wait(&sm.pt_empty, (ac - 1) & 1, abort_flag, P.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++sc;
+      tc_fence_after();
+      const bool msk = (P.causal && it == j) || ((it + 1) * kTile > P.N) || !key_ok;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t rs[32], rp[32];
+        tmem_ld32x2(t_lane + kColS + ch * 32, rs, t_lane + kColDP + ch * 32, rp);
+        if (ch == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_empty);
+        }
+        uint32_t wp[16], wd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 tv = *reinterpret_cast<const float4*>(&sm.tau[slot][ch * 32 + e]);
+          const float4 dv = *reinterpret_cast<const float4*>(&sm.delta[slot][ch * 32 + e]);
+          const float taus[4] = {tv.x, tv.y, tv.z, tv.w};
+          const float dels[4] = {dv.x, dv.y, dv.z, dv.w};
+          float pp[4], dd[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float tt = fmaf(__uint_as_float(rs[e + u]), P.c, -taus[u]);
+            if (msk) {
+              const int row = it * kTile + ch * 32 + e + u;
+              const bool ok_e = key_ok && row < P.N && (!P.causal || key <= row);
+              if (!ok_e) tt = -1.0f;
+            }
+            const float tp = fmaxf(tt, 0.0f);
+            const float g = ALPHA2 ? (tt > 0.f ? 1.f : 0.f) : tp;
+            pp[u] = ALPHA2 ? tp : tp * tp;
+            dd[u] = g * (__uint_as_float(rp[e + u]) - dels[u]);
+          }
+          __half2 a0 = __floats2half2_rn(pp[0], pp[1]);
+          __half2 a1 = __floats2half2_rn(pp[2], pp[3]);
+          __half2 b0 = __floats2half2_rn(dd[0], dd[1]);
+          __half2 b1 = __floats2half2_rn(dd[2], dd[3]);
+          wp[e / 2] = *reinterpret_cast<uint32_t*>(&a0);
+          wp[e / 2 + 1] = *reinterpret_cast<uint32_t*>(&a1);
+          wd[e / 2] = *reinterpret_cast<uint32_t*>(&b0);
+          wd[e / 2 + 1] = *reinterpret_cast<uint32_t*>(&b1);
+        }
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+          const uint32_t off = sw128_chunk_offset(kl, ch * 4 + qd);
+          *reinterpret_cast<uint4*>(pt_base + off) =
+              make_uint4(wp[4 * qd], wp[4 * qd + 1], wp[4 * qd + 2], wp[4 * qd + 3]);
+          *reinterpret_cast<uint4*>(ds_base + off) =
+              make_uint4(wd[4 * qd], wd[4 * qd + 1], wd[4 * qd + 2], wd[4 * qd + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.pt_full);
+      ++ac;
+    }
+    if (ok && n > 0) {
+      ok = mbar_wait(&sm.acc_full, 0, abort_flag, P.status);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    tc_fence_after();
+    const size_t base = (static_cast<size_t>(bh) * P.N + key) * D;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t col = which == 0 ? kColDV : kColDK;
+      const float scale = which == 0 ? 1.0f : P.inv_sqrt_d;
+      __nv_bfloat16* dst_row = (which == 0 ? P.dv : P.dk) + base;
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t r[32];
+        if (ok && n > 0) {
+          tmem_ld32(t_lane + col + ch * 32, r);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+        if (key_ok) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * scale,
+                                                            __uint_as_float(r[2 * e + 1]) * scale);
+            w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 32);
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd)
+            dst[qd] = make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (sm.abort_flag) {
+    if (warp == 0 && lane == 0) {
+      mbar_wait(&sm.kv_full, 0, nullptr, nullptr);
+      for (uint32_t s = 0; s < NS; ++s)
+        if (qc > s) mbar_wait(&sm.q_full[s], ((qc - 1 - s) / NS) & 1, nullptr, nullptr);
+    }
+    if (warp == 1 && lane == 0) {
+      mma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, nullptr, nullptr);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace entmax

@@ -1,0 +1,96 @@
+// Shared constants and small device helpers of the alpha-entmax kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace entmax {
+
+constexpr int kTile = 128;                   // compute tile: 128 query rows x 128 keys
+constexpr int kThreads = 192;                // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kEpiThreads = 128;
+constexpr int kMaxN = 262144;
+constexpr int kMaxTiles = kMaxN / kTile;     // 2048 tiles per row
+constexpr int kMaxMaskWords = kMaxN / 64 / 32;  // words per mask row at block 64
+constexpr int kSlabBytes = kTile * 128;      // one [128 rows][128 B] swizzled slab
+constexpr int kNB = 8;                       // histogram bins per unit of s
+constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23
+constexpr uint32_t kMagicBits = 0x4B400000u; // bit pattern of kMagic
+
+enum PassKind : int { PASS_HIST = 0, PASS_REFINE = 1, PASS_PV = 2, PASS_DONE = 3 };
+
+// Work counters kept in the workspace right after the status word (uint64 each).
+enum Counter : int {
+  CNT_HIST_TILES = 0,    // forward: key tiles visited by histogram passes
+  CNT_REFINE_TILES = 1,  // forward: key tiles visited by refinement passes
+  CNT_PV_TILES = 2,      // forward: key tiles visited by the P.V pass
+  CNT_REFINE_PASSES = 3, // forward: refinement passes, summed over 128-row tiles
+  CNT_ROW_TILES = 4,     // backward: key tiles per pass of the row kernel
+  CNT_COL_TILES = 5,     // backward: query tiles visited by the column kernel
+  CNT_COUNT = 8
+};
+
+// Named barrier over the four epilogue warps only (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// 64-bit left shift with the PTX clamp rule: a shift amount >= 64 (including
+// "negative" amounts seen as huge unsigned values) yields 0.
+__device__ __forceinline__ uint64_t shl64(uint64_t x, uint32_t sh) {
+  uint64_t r;
+  asm("shl.b64 %0, %1, %2;" : "=l"(r) : "l"(x), "r"(sh));
+  return r;
+}
+
+// Offset (in 128-element rows) of the tile-max record of (row tile i, key tile
+// j) of head bh.  Causal problems store only the lower triangle j <= i.
+__device__ __forceinline__ size_t tmax_index(int bh, int i, int j, int tr, int tc, int causal) {
+  const size_t per = causal ? static_cast<size_t>(tr) * (tr + 1) / 2
+                            : static_cast<size_t>(tr) * tc;
+  const size_t idx = causal ? static_cast<size_t>(i) * (i + 1) / 2 + j
+                            : static_cast<size_t>(i) * tc + j;
+  return (static_cast<size_t>(bh) * per + idx) * kTile;
+}
+
+// Byte offset, inside a 128-byte-swizzled K-major tile made of [128 rows][64
+// bf16] slabs, of the 16-byte chunk holding elements [8c, 8c+8) of row `row`
+// (element index counted across slabs).  The tensor core and TMA apply the
+// same XOR of address bits [4,7) with bits [7,10).
+__device__ __forceinline__ uint32_t sw128_chunk_offset(int row, int chunk16) {
+  const int slab = chunk16 >> 3;
+  const int c = chunk16 & 7;
+  return static_cast<uint32_t>(slab * kSlabBytes + row * 128 + ((c ^ (row & 7)) << 4));
+}
+
+// Warp-parallel compaction of the set bits of flags[0, nwords) into a sorted
+// tile list (find-first-set / popcount traversal).  Clears the flags it read.
+// Executed by one full warp; returns the number of tiles.
+__device__ __forceinline__ int compact_tiles(uint32_t* flags, int nwords, uint16_t* tiles) {
+  const int lane = threadIdx.x & 31;
+  int total = 0;
+  for (int base = 0; base < nwords; base += 32) {
+    const int w = base + lane;
+    uint32_t word = (w < nwords) ? flags[w] : 0u;
+    if (w < nwords) flags[w] = 0u;
+    const int cnt = __popc(word);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int pos = total + incl - cnt;
+    while (word) {
+      const int b = __ffs(word) - 1;
+      tiles[pos++] = static_cast<uint16_t>(w * 32 + b);
+      word &= word - 1u;
+    }
+    total += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return total;
+}
+
+}  // namespace entmax

@@ -1,0 +1,395 @@
+// Host side of the C ABI declared in include/entmax_attn.h: argument checks,
+// workspace layout, TMA tensor maps and kernel launches.  No memory is
+// allocated here; every buffer belongs to the caller.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <algorithm>
+#include <mutex>
+
+#include "entmax_attn.h"
+#include "fwd.cuh"
+#include "bwd.cuh"
+
+using namespace entmax;
+
+namespace {
+
+// ------------------------------------------------------------ workspace layout
+struct WsLayout {
+  size_t status = 0;     // uint32 status word (+ padding)
+  size_t tmax = 0;       // fp16 per-(row, key tile) maxima of s
+  size_t tilemask = 0;   // uint32 [BH][T][ceil(T/32)] 128-granularity mask
+  size_t tilemaskT = 0;  // uint32 [BH][T][ceil(T/32)] its transpose
+  size_t delta = 0;      // float [BH][N]
+  size_t half_copies = 0;  // fp16 copies of q, k, v, dout for the backward
+  size_t total = 0;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+WsLayout ws_layout(int B, int H, int N, int D, int causal) {
+  WsLayout L;
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t t = (static_cast<size_t>(N) + kTile - 1) / kTile;
+  const size_t tiles = causal ? t * (t + 1) / 2 : t * t;
+  const size_t words = (t + 31) / 32;
+  size_t off = 256;
+  L.tmax = off;
+  off = align256(off + bh * tiles * kTile * sizeof(__half));
+  L.tilemask = off;
+  off = align256(off + bh * t * words * sizeof(uint32_t));
+  L.tilemaskT = off;
+  off = align256(off + bh * t * words * sizeof(uint32_t));
+  L.delta = off;
+  off = align256(off + bh * static_cast<size_t>(N) * sizeof(float));
+  L.half_copies = off;
+  off = align256(off + 4 * bh * static_cast<size_t>(N) * D * sizeof(__half));
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------ argument checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int H, int N, int D, int dtype, float alpha, int block) {
+  if (B < 1 || H < 1 || N < 1 || N > kMaxN) return ENTMAX_E_SHAPE;
+  if (static_cast<long long>(B) * H * ((N + kTile - 1) / kTile) > 0x7fffffffLL) return ENTMAX_E_SHAPE;
+  if (D != 64 && D != 128) return ENTMAX_E_UNSUPPORTED;
+  if (dtype != ENTMAX_DTYPE_BF16) return ENTMAX_E_UNSUPPORTED;
+  if (block != 64 && block != 128) return ENTMAX_E_UNSUPPORTED;
+  if (!(alpha == 1.5f || alpha == 2.0f)) return ENTMAX_E_ALPHA;
+  return ENTMAX_OK;
+}
+
+// ------------------------------------------------------------ TMA tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [BH][N][D] tensor as a 3-D map {D, N, BH}; box {64 bf16 = 128 B, 128 rows, 1};
+// 128-byte swizzle so tiles land in the layout the UMMA descriptors describe.
+// Rows past N read as zeros.
+bool make_map(CUtensorMap* m, const void* base, int BH, int N, int D,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  auto enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTile), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ profiling aid
+// Per calling thread: when enabled, fwd/bwd record CUDA events on their stream
+// around each kernel; entmax_attn_profile_read() turns them into milliseconds.
+enum : int { EV_FWD0, EV_FWD1, EV_BWD0, EV_BWD_CONV, EV_BWD_MASK, EV_BWD_ROW, EV_BWD_COL, EV_COUNT };
+struct Profiler {
+  bool on = false;
+  bool created = false;
+  cudaEvent_t ev[EV_COUNT] = {};
+};
+thread_local Profiler g_prof;
+
+void prof_mark(int idx, cudaStream_t st) {
+  if (g_prof.on && g_prof.created) cudaEventRecord(g_prof.ev[idx], st);
+}
+
+template <typename Kernel>
+bool set_smem(Kernel k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bytes)) == cudaSuccess;
+}
+
+template <int D, int NS, bool A2>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const FwdParams& p, cudaStream_t st) {
+  auto kern = entmax_fwd_kernel<D, NS, A2>;
+  constexpr size_t smem = fwd_smem_bytes<D, NS>();
+  static_assert(smem <= 232448, "forward kernel shared memory");
+  static bool attr_ok = set_smem(kern, smem);
+  if (!attr_ok) return ENTMAX_E_CUDA;
+  const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.tr);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
+}
+
+template <int D, int NSK, int NSV, bool A2>
+int launch_bwd_row(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const CUtensorMap& mdo, const BwdParams& p, cudaStream_t st) {
+  auto kern = entmax_bwd_row_kernel<D, NSK, NSV, A2>;
+  constexpr size_t smem = bwd_row_smem_bytes<D, NSK, NSV>();
+  static_assert(smem <= 232448, "bwd row kernel shared memory");
+  static bool attr_ok = set_smem(kern, smem);
+  if (!attr_ok) return ENTMAX_E_CUDA;
+  const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.T);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
+}
+
+template <int D, int NS, bool A2>
+int launch_bwd_col(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const CUtensorMap& mdo, const BwdParams& p, cudaStream_t st) {
+  auto kern = entmax_bwd_col_kernel<D, NS, A2>;
+  constexpr size_t smem = bwd_col_smem_bytes<D, NS>();
+  static_assert(smem <= 232448, "bwd column kernel shared memory");
+  static bool attr_ok = set_smem(kern, smem);
+  if (!attr_ok) return ENTMAX_E_CUDA;
+  const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.T);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
+}
+
+}  // namespace
+
+// ============================================================== C ABI
+extern "C" {
+
+int entmax_attn_mask_words(int N, int block) {
+  if (N < 1 || N > kMaxN) return ENTMAX_E_SHAPE;
+  if (block != 64 && block != 128) return ENTMAX_E_UNSUPPORTED;
+  const int tb = (N + block - 1) / block;
+  return (tb + 31) / 32;
+}
+
+size_t entmax_attn_workspace_size(int B, int H, int N, int D, int block, int causal) {
+  if (B < 1 || H < 1 || N < 1 || N > kMaxN) return 0;
+  if ((D != 64 && D != 128) || (block != 64 && block != 128)) return 0;
+  return ws_layout(B, H, N, D, causal ? 1 : 0).total;
+}
+
+int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int D,
+                    int dtype, float alpha, int causal, int block, int max_iter, void* out,
+                    float* tau, uint32_t* mask, float* tau_trace, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out || !tau || !mask || !workspace) return ENTMAX_E_NULL;
+  int rc = check_common(B, H, N, D, dtype, alpha, block);
+  if (rc != ENTMAX_OK) return rc;
+  if (max_iter < 0 || max_iter > ENTMAX_MAX_ITER) return ENTMAX_E_MAXITER;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(tau) ||
+      !aligned16(mask) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return ENTMAX_E_ALIGN;
+  const WsLayout L = ws_layout(B, H, N, D, causal ? 1 : 0);
+  if (workspace_bytes < L.total) return ENTMAX_E_WORKSPACE;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
+    return ENTMAX_E_CUDA;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // status word + work counters live in the first 256 bytes
+  if (cudaMemsetAsync(ws + L.status, 0, 8 + CNT_COUNT * sizeof(unsigned long long), st) != cudaSuccess)
+    return ENTMAX_E_CUDA;
+
+  FwdParams p{};
+  p.BH = BH;
+  p.N = N;
+  p.tr = (N + kTile - 1) / kTile;
+  p.tc = p.tr;
+  p.causal = causal ? 1 : 0;
+  p.block = block;
+  p.mask_rows = (N + block - 1) / block;
+  p.mask_words = (p.mask_rows + 31) / 32;
+  p.max_iter = max_iter;
+  p.c = (alpha - 1.0f) / std::sqrt(static_cast<float>(D));
+  p.cN = p.c * static_cast<float>(kNB);
+  p.slim = 2097152.0f / p.cN;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.tau = tau;
+  p.mask = mask;
+  p.tau_trace = tau_trace;
+  p.tmax = reinterpret_cast<__half*>(ws + L.tmax);
+  p.status = reinterpret_cast<uint32_t*>(ws + L.status);
+  p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
+
+  const bool a2 = alpha == 2.0f;
+  prof_mark(EV_FWD0, st);
+  if (D == 64) {
+    rc = a2 ? launch_fwd<64, 3, true>(mq, mk, mv, p, st) : launch_fwd<64, 3, false>(mq, mk, mv, p, st);
+  } else {
+    rc = a2 ? launch_fwd<128, 2, true>(mq, mk, mv, p, st) : launch_fwd<128, 2, false>(mq, mk, mv, p, st);
+  }
+  prof_mark(EV_FWD1, st);
+  return rc;
+}
+
+int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                    const float* tau, const uint32_t* mask, int B, int H, int N, int D,
+                    int dtype, float alpha, int causal, int block, void* dq, void* dk, void* dv,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dout || !tau || !mask || !dq || !dk || !dv || !workspace)
+    return ENTMAX_E_NULL;
+  int rc = check_common(B, H, N, D, dtype, alpha, block);
+  if (rc != ENTMAX_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(tau) ||
+      !aligned16(mask) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return ENTMAX_E_ALIGN;
+  const WsLayout L = ws_layout(B, H, N, D, causal ? 1 : 0);
+  if (workspace_bytes < L.total) return ENTMAX_E_WORKSPACE;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status_word = reinterpret_cast<uint32_t*>(ws + L.status);
+  unsigned long long* counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
+  if (cudaMemsetAsync(counters + CNT_ROW_TILES, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+    return ENTMAX_E_CUDA;
+  prof_mark(EV_BWD0, st);
+  const size_t elems = static_cast<size_t>(BH) * N * D;
+  __half* h16[4];
+  const void* srcs[4] = {q, k, v, dout};
+  for (int a = 0; a < 4; ++a) {
+    h16[a] = reinterpret_cast<__half*>(ws + L.half_copies) + a * elems;
+    const size_t n8 = elems / 8;  // D is a multiple of 8
+    const int grid = static_cast<int>(std::min<size_t>((n8 + 255) / 256, 148 * 8));
+    to_fp16_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(srcs[a]), h16[a], n8,
+                                         status_word);
+  }
+  if (cudaGetLastError() != cudaSuccess) return ENTMAX_E_CUDA;
+  prof_mark(EV_BWD_CONV, st);
+  CUtensorMap mq, mk, mv, mdo;
+  const auto f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  if (!make_map(&mq, h16[0], BH, N, D, f16) || !make_map(&mk, h16[1], BH, N, D, f16) ||
+      !make_map(&mv, h16[2], BH, N, D, f16) || !make_map(&mdo, h16[3], BH, N, D, f16))
+    return ENTMAX_E_CUDA;
+
+  const int T = (N + kTile - 1) / kTile;
+  const int wt = (T + 31) / 32;
+  const int mask_rows = (N + block - 1) / block;
+  const int mask_words = (mask_rows + 31) / 32;
+  uint32_t* tm = reinterpret_cast<uint32_t*>(ws + L.tilemask);
+  uint32_t* tmt = reinterpret_cast<uint32_t*>(ws + L.tilemaskT);
+  {
+    const long long words = static_cast<long long>(BH) * T * wt;
+    const int threads = 256;
+    const int grid = static_cast<int>(std::min<long long>((words + threads - 1) / threads, 148 * 16));
+    tile_mask_kernel<<<grid, threads, 0, st>>>(mask, tm, BH, T, block, mask_rows, mask_words);
+    tile_mask_t_kernel<<<grid, threads, 0, st>>>(tm, tmt, BH, T);
+    if (cudaGetLastError() != cudaSuccess) return ENTMAX_E_CUDA;
+  }
+  prof_mark(EV_BWD_MASK, st);
+
+  BwdParams p{};
+  p.BH = BH;
+  p.N = N;
+  p.T = T;
+  p.wt = wt;
+  p.causal = causal ? 1 : 0;
+  p.c = (alpha - 1.0f) / std::sqrt(static_cast<float>(D));
+  p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(D));
+  p.tau = tau;
+  p.delta = reinterpret_cast<float*>(ws + L.delta);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.status = status_word;
+  p.counters = counters;
+
+  const bool a2 = alpha == 2.0f;
+  BwdParams prow = p;
+  prow.tm = tm;
+  BwdParams pcol = p;
+  pcol.tm = tmt;
+  if (D == 64) {
+    rc = a2 ? launch_bwd_row<64, 3, 2, true>(mq, mk, mv, mdo, prow, st)
+            : launch_bwd_row<64, 3, 2, false>(mq, mk, mv, mdo, prow, st);
+    if (rc != ENTMAX_OK) return rc;
+    prof_mark(EV_BWD_ROW, st);
+    rc = a2 ? launch_bwd_col<64, 3, true>(mq, mk, mv, mdo, pcol, st)
+            : launch_bwd_col<64, 3, false>(mq, mk, mv, mdo, pcol, st);
+  } else {
+    rc = a2 ? launch_bwd_row<128, 2, 1, true>(mq, mk, mv, mdo, prow, st)
+            : launch_bwd_row<128, 2, 1, false>(mq, mk, mv, mdo, prow, st);
+    if (rc != ENTMAX_OK) return rc;
+    prof_mark(EV_BWD_ROW, st);
+    rc = a2 ? launch_bwd_col<128, 1, true>(mq, mk, mv, mdo, pcol, st)
+            : launch_bwd_col<128, 1, false>(mq, mk, mv, mdo, pcol, st);
+  }
+  prof_mark(EV_BWD_COL, st);
+  return rc;
+}
+
+int entmax_attn_status(const void* workspace, void* stream, uint32_t* status) {
+  if (!workspace || !status) return ENTMAX_E_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ENTMAX_E_CUDA;
+  if (cudaMemcpy(status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ENTMAX_E_CUDA;
+  return ENTMAX_OK;
+}
+
+int entmax_attn_counters(const void* workspace, void* stream, unsigned long long* counters,
+                         int n) {
+  if (!workspace || !counters) return ENTMAX_E_NULL;
+  if (n < 1 || n > CNT_COUNT) return ENTMAX_E_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ENTMAX_E_CUDA;
+  if (cudaMemcpy(counters, static_cast<const uint8_t*>(workspace) + 8,
+                 n * sizeof(unsigned long long), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ENTMAX_E_CUDA;
+  return ENTMAX_OK;
+}
+
+int entmax_attn_profile(int enable) {
+  if (enable && !g_prof.created) {
+    for (int e = 0; e < EV_COUNT; ++e)
+      if (cudaEventCreate(&g_prof.ev[e]) != cudaSuccess) return ENTMAX_E_CUDA;
+    g_prof.created = true;
+  }
+  g_prof.on = enable != 0;
+  return ENTMAX_OK;
+}
+
+int entmax_attn_profile_read(float* ms, int n) {
+  if (!ms) return ENTMAX_E_NULL;
+  if (n < 1 || n > 5) return ENTMAX_E_SHAPE;
+  if (!g_prof.created) return ENTMAX_E_CUDA;
+  const int pairs[5][2] = {{EV_FWD0, EV_FWD1}, {EV_BWD0, EV_BWD_CONV}, {EV_BWD_CONV, EV_BWD_MASK},
+                           {EV_BWD_MASK, EV_BWD_ROW}, {EV_BWD_ROW, EV_BWD_COL}};
+  for (int a = 0; a < n; ++a) {
+    if (cudaEventSynchronize(g_prof.ev[pairs[a][1]]) != cudaSuccess) return ENTMAX_E_CUDA;
+    if (cudaEventElapsedTime(&ms[a], g_prof.ev[pairs[a][0]], g_prof.ev[pairs[a][1]]) != cudaSuccess)
+      return ENTMAX_E_CUDA;
+  }
+  return ENTMAX_OK;
+}
+
+const char* entmax_attn_error_string(int code) {
+  switch (code) {
+    case ENTMAX_OK: return "success";
+    case ENTMAX_E_NULL: return "a required pointer is NULL";
+    case ENTMAX_E_ALIGN: return "a tensor pointer is not 16-byte aligned (workspace: 256-byte)";
+    case ENTMAX_E_SHAPE: return "B, H or N out of range";
+    case ENTMAX_E_UNSUPPORTED: return "head dim, dtype or block size not supported";
+    case ENTMAX_E_ALPHA: return "alpha not supported (1.5 or 2.0)";
+    case ENTMAX_E_WORKSPACE: return "workspace smaller than entmax_attn_workspace_size()";
+    case ENTMAX_E_CUDA: return "a CUDA call failed";
+    case ENTMAX_E_MAXITER: return "max_iter out of range";
+    default: return "unknown error code";
+  }
+}
+
+}  // extern "C"

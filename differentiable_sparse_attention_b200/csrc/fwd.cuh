@@ -1,0 +1,681 @@
+// Forward alpha-entmax attention kernel for sm_100a (bf16 inputs, f32 accumulate).
+//
+// One CTA owns a 128-row query tile of one (batch, head).  Warp 0 streams
+// K/V tiles with TMA, warp 1 issues tcgen05 MMAs into TMEM, warps 2-5 (one
+// thread per query row) run the epilogues.  The CTA walks a sequence of passes
+// over key tiles, each pass driven by a tile list in shared memory:
+//
+//   HIST    every visible key tile: S = Q K^T, running row max, 8-bin
+//           histogram of the scores in the unit window below the max
+//           (AdaSplash-2 zh §2.1 / it §2A / ja §2.1 / es §2A), and a rounded-up
+//           per-(row, tile) score maximum kept in the workspace.  The reduced
+//           histogram problem gives tau_h with tau* - h <= tau_h <= tau*
+//           (Proposition 1 of the paper, as the summaries state it).
+//   REFINE  1..max_iter safeguarded steps from tau_h (zh §2.2, it §2B, ja §2.2,
+//           es §2B): Halley for alpha = 1.5, Newton for alpha = 2, bisection
+//           whenever the step leaves the bracket [lo, hi].  Only tiles whose
+//           recorded maximum exceeds the row's lower bound lo are visited:
+//           tiles entirely below lo <= tau* contribute nothing.
+//   PV      the surviving tiles: p = [s - tau]_+^(1/(alpha-1)) written to SMEM as
+//           bf16, O += P V on the tensor cores, and the bit-packed block mask
+//           (32 blocks per uint32 word, zh §2.3) of blocks holding a p > 0.
+#pragma once
+
+#include "common.cuh"
+
+namespace entmax {
+
+struct FwdParams {
+  int BH, N, tr, tc;         // heads x batch, sequence length, 128-tiles per row / column
+  int causal;
+  int block;                 // mask block size, 64 or 128
+  int mask_rows, mask_words; // ceil(N / block), words per mask row
+  int max_iter;
+  float c;                   // (alpha - 1) / sqrt(D): s = c * (q . k)
+  float cN;                  // c * kNB (exact: kNB is a power of two)
+  float slim;                // 2^21 / cN: scores beyond are outside the exact binning range
+  __nv_bfloat16* out;
+  float* tau;
+  uint32_t* mask;
+  float* tau_trace;          // nullable, [max_iter + 1][BH][N]
+  __half* tmax;              // workspace: per-(row, key tile) maxima of s, rounded up
+  uint32_t* status;          // workspace word 0
+  unsigned long long* counters;  // workspace, CNT_* work counters
+};
+
+template <int D, int NS>
+struct FwdSmem {
+  __nv_bfloat16 q[kTile * D];       // D/64 swizzled slabs
+  __nv_bfloat16 k[NS][kTile * D];
+  __nv_bfloat16 v[NS][kTile * D];
+  __nv_bfloat16 p[kTile * kTile];   // P tile, K-major (K = keys), 2 slabs
+  uint64_t q_full;
+  uint64_t k_full[NS], k_empty[NS];
+  uint64_t v_full[NS], v_empty[NS];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full, p_empty, o_full, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int ctl_kind, ctl_n, ctl_iter;
+  int not_converged;
+  uint32_t flags[kMaxTiles / 32];
+  uint32_t maskw[2][kMaxMaskWords];
+  uint16_t tiles[kMaxTiles];
+};
+
+template <int D, int NS>
+constexpr size_t fwd_smem_bytes() {
+  return sizeof(FwdSmem<D, NS>) + 1024;  // + slack for 1024-byte alignment
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+template <int D, int NS, bool ALPHA2>
+__global__ void __launch_bounds__(kThreads, 1)
+    entmax_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const FwdParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  FwdSmem<D, NS>& sm = *reinterpret_cast<FwdSmem<D, NS>*>(align1024(smem_raw));
+  constexpr int kSlabs = D / 64;
+  constexpr uint32_t kTileBytes = kTile * D * 2;
+  constexpr uint32_t kIdescS = make_idesc(kTile, kTile, 1, 1, 0, 0);  // Q (K-major) x K (K-major)
+  constexpr uint32_t kIdescPV = make_idesc(kTile, D, 1, 1, 0, 1);     // P (K-major) x V (MN-major)
+  constexpr uint32_t kColO = 256;                                     // TMEM: S0, S1, O
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // Work unit: the latest (longest causal) row tiles first.
+  const int i = P.tr - 1 - static_cast<int>(blockIdx.x) / P.BH;
+  const int bh = static_cast<int>(blockIdx.x) % P.BH;
+  const int ntc = P.causal ? (i + 1) : P.tc;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.s_empty[s], 4);
+    }
+    mbar_init(&sm.p_full, 4);
+    mbar_init(&sm.p_empty, 1);
+    mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    sm.not_converged = 0;
+    sm.ctl_kind = PASS_HIST;
+    sm.ctl_n = ntc;
+    sm.ctl_iter = 0;
+    fence_mbar_init();
+  }
+  for (int w = threadIdx.x; w < kMaxTiles / 32; w += kThreads) sm.flags[w] = 0u;
+  for (int w = threadIdx.x; w < 2 * kMaxMaskWords; w += kThreads) (&sm.maskw[0][0])[w] = 0u;
+  for (int t = threadIdx.x; t < ntc; t += kThreads) sm.tiles[t] = static_cast<uint16_t>(t);
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  // -------- role state that lives across passes
+  uint32_t kc = 0, vc = 0, sc = 0, pc = 0;   // K loads, V loads, S tiles, PV tiles
+  bool q_issued = false, q_waited = false;
+
+  // epilogue (one query row per thread)
+  const int quad = warp & 3;
+  const int rl = quad * 32 + lane;
+  const int row = i * kTile + rl;
+  const bool row_ok = (warp >= 2) && row < P.N;
+  const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+  const int n_valid = P.causal ? min(row + 1, P.N) : P.N;
+  float m_raw = -INFINITY;                 // running max of q.k (raw units)
+  int gtop = 0;                            // grid index floor(kNB * s) of the max
+  bool gtop_set = false;
+  uint32_t cnt[kNB + 1];
+#pragma unroll
+  for (int b = 0; b <= kNB; ++b) cnt[b] = 0u;
+  float vclamp = -P.slim;                  // scores are clamped to >= vclamp before binning
+  uint32_t cbase = 0u;
+  double lo = 0.0, hi = 0.0;               // bracket of tau*
+  float tau_c = 0.0f;                      // current evaluation point / final tau
+  int iter = 0;
+  bool row_done = false;                   // threshold certified exact
+  float rowsum = 0.0f;
+
+  auto trace_store = [&](int it, float val) {
+    if (P.tau_trace != nullptr && row_ok)
+      P.tau_trace[(static_cast<size_t>(it) * P.BH + bh) * P.N + row] = val;
+  };
+
+  // Per-element validity only matters on the diagonal tile (causal) and on
+  // the ragged last key tile.
+  auto needs_mask = [&](int j) {
+    return (P.causal && j == i) || ((j + 1) * kTile > P.N);
+  };
+  auto apply_mask = [&](float (&v)[32], int j, int ch) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int col = j * kTile + ch * 32 + e;
+      const bool ok = col < P.N && (!P.causal || col <= row);
+      v[e] = ok ? v[e] : -INFINITY;
+    }
+  };
+
+  for (;;) {
+    __syncthreads();
+    const int kind = sm.ctl_kind;
+    const int n = sm.ctl_n;
+    const int aborted = sm.abort_flag;
+    __syncthreads();
+    if (aborted || kind == PASS_DONE) break;
+
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        bool ok = true;
+        if (!q_issued) {
+          q_issued = true;
+          mbar_expect_tx(&sm.q_full, kTileBytes);
+#pragma unroll
+          for (int s = 0; s < kSlabs; ++s)
+            tma_load_3d(sm.q + s * kTile * 64, &tm_q, &sm.q_full, s * 64, i * kTile, bh);
+        }
+        for (int t = 0; t < n && ok; ++t) {
+          const int j = sm.tiles[t];
+          {
+            const uint32_t slot = kc % NS, use = kc / NS;
+            if (use > 0 && !mbar_wait(&sm.k_empty[slot], (use - 1) & 1, abort_flag, P.status)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(&sm.k_full[slot], kTileBytes);
+#pragma unroll
+            for (int s = 0; s < kSlabs; ++s)
+              tma_load_3d(sm.k[slot] + s * kTile * 64, &tm_k, &sm.k_full[slot], s * 64,
+                          j * kTile, bh);
+            ++kc;
+          }
+          if (kind == PASS_PV) {
+            const uint32_t slot = vc % NS, use = vc / NS;
+            if (use > 0 && !mbar_wait(&sm.v_empty[slot], (use - 1) & 1, abort_flag, P.status)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(&sm.v_full[slot], kTileBytes);
+#pragma unroll
+            for (int s = 0; s < kSlabs; ++s)
+              tma_load_3d(sm.v[slot] + s * kTile * 64, &tm_v, &sm.v_full[slot], s * 64,
+                          j * kTile, bh);
+            ++vc;
+          }
+        }
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        bool ok = true;
+        if (!q_waited) {
+          q_waited = true;
+          ok = mbar_wait(&sm.q_full, 0, abort_flag, P.status);
+        }
+        const uint32_t q_addr = smem_u32(sm.q);
+        auto issue_s = [&]() -> bool {
+          const uint32_t slot = kc % NS;
+          if (!mbar_wait(&sm.k_full[slot], (kc / NS) & 1, abort_flag, P.status)) return false;
+          const uint32_t sb = sc & 1, use = sc >> 1;
+          if (use > 0 && !mbar_wait(&sm.s_empty[sb], (use - 1) & 1, abort_flag, P.status))
+            return false;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sm.k[slot]);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+            mma_f16_ss(tmem + sb * kTile, smem_desc_sw128(q_addr + off, 16, 1024),
+                       smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&sm.s_full[sb]);
+          mma_commit(&sm.k_empty[slot]);
+          ++kc;
+          ++sc;
+          return true;
+        };
+        auto issue_pv = [&]() -> bool {
+          if (!mbar_wait(&sm.p_full, pc & 1, abort_flag, P.status)) return false;
+          const uint32_t slot = vc % NS;
+          if (!mbar_wait(&sm.v_full[slot], (vc / NS) & 1, abort_flag, P.status)) return false;
+          tc_fence_after();
+          const uint32_t p_addr = smem_u32(sm.p);
+          const uint32_t v_addr = smem_u32(sm.v[slot]);
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint32_t a_off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+            const uint32_t b_off = kk * 16 * 128;  // 16 keys of 128-byte rows
+            mma_f16_ss(tmem + kColO, smem_desc_sw128(p_addr + a_off, 16, 1024),
+                       smem_desc_sw128(v_addr + b_off, kSlabBytes, 1024), kIdescPV,
+                       (pc > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&sm.v_empty[slot]);
+          mma_commit(&sm.p_empty);
+          ++vc;
+          ++pc;
+          return true;
+        };
+        if (ok) {
+          if (kind != PASS_PV) {
+            for (int t = 0; t < n && ok; ++t) ok = issue_s();
+          } else {
+            for (int t = 0; t <= n && ok; ++t) {
+              if (t < n) ok = issue_s();
+              if (ok && t > 0) ok = issue_pv();
+            }
+            if (ok) mma_commit(&sm.o_full);
+          }
+        }
+      }
+      __syncwarp();
+    } else {
+      // ------------------------------------------------------------ epilogue
+      bool ok = true;
+      double F0 = 0.0, F1 = 0.0, F2 = 0.0;  // refinement sums at tau_c
+      float Tmin = INFINITY;                // smallest positive s - tau_c
+      if (kind == PASS_PV) rowsum = 0.0f;
+      for (int t = 0; t < n; ++t) {
+        const int j = sm.tiles[t];
+        const uint32_t cur = sc++;
+        const uint32_t sb = cur & 1;
+        ok = mbar_wait(&sm.s_full[sb], (cur >> 1) & 1, abort_flag, P.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const bool msk = needs_mask(j);
+        const uint32_t t_s = t_lane + sb * kTile;
+
+        if (kind == PASS_HIST) {
+          float tile_max = -INFINITY;
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(t_s + ch * 32, r);
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+            if (msk) apply_mask(v, j, ch);
+            float cm = v[0];
+#pragma unroll
+            for (int e = 1; e < 32; ++e) cm = fmaxf(cm, v[e]);
+            tile_max = fmaxf(tile_max, cm);
+            if (cm > -INFINITY) {
+              const int gc = static_cast<int>(
+                  __float_as_uint(__fmaf_rd(fmaxf(cm, -P.slim), P.cN, kMagic)) - kMagicBits);
+              if (!gtop_set || gc > gtop) {
+                const int delta = gtop_set ? gc - gtop : kNB + 1;
+                if (delta > kNB) {
+#pragma unroll
+                  for (int b = 0; b <= kNB; ++b) cnt[b] = 0u;
+                } else {
+                  for (int d = 0; d < delta; ++d) {
+#pragma unroll
+                    for (int b = 0; b < kNB; ++b) cnt[b] = cnt[b + 1];
+                    cnt[kNB] = 0u;
+                  }
+                }
+                gtop = gc;
+                gtop_set = true;
+                // Scores below the window are clamped to grid index <= base - 1,
+                // whose shift amount is "negative" and adds nothing.
+                vclamp = (static_cast<float>(gtop - kNB) - 1.5f) / P.cN;
+                cbase = 0u - 7u * (kMagicBits + static_cast<uint32_t>(gtop - kNB));
+              }
+              // 9 bins in 7-bit lanes of one 64-bit word (<= 32 counts per chunk):
+              // bin b of a score is floor(kNB * s) - (gtop - kNB), exact via a
+              // round-down FMA against 1.5 * 2^23.
+              uint64_t packed = 0;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const float u = __fmaf_rd(fmaxf(v[e], vclamp), P.cN, kMagic);
+                const uint32_t sh = __float_as_uint(u) * 7u + cbase;
+                packed += shl64(1ull, sh);
+              }
+#pragma unroll
+              for (int b = 0; b <= kNB; ++b)
+                cnt[b] += static_cast<uint32_t>(packed >> (7 * b)) & 127u;
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+          m_raw = fmaxf(m_raw, tile_max);
+          const float rec = row_ok ? tile_max * P.c : -INFINITY;
+          P.tmax[tmax_index(bh, i, j, P.tr, P.tc, P.causal) + rl] = __float2half_ru(rec);
+        } else if (kind == PASS_REFINE) {
+          float f0 = 0.f, f1 = 0.f, f2 = 0.f, tmin = INFINITY;
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(t_s + ch * 32, r);
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+            if (msk) apply_mask(v, j, ch);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float tt = fmaf(v[e], P.c, -tau_c);
+              const bool in = tt > 0.0f;
+              const float tp = fmaxf(tt, 0.0f);
+              tmin = in ? fminf(tmin, tt) : tmin;
+              if (ALPHA2) {
+                f0 += tp;
+                f1 += in ? 1.0f : 0.0f;
+              } else {
+                f0 = fmaf(tp, tp, f0);
+                f1 += tp;
+                f2 += in ? 1.0f : 0.0f;
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+          F0 += f0;
+          F1 += f1;
+          F2 += f2;
+          Tmin = fminf(Tmin, tmin);
+        } else {  // PASS_PV
+          const uint32_t cur_p = pc++;
+          if (cur_p > 0) {
+            ok = mbar_wait(&sm.p_empty, (cur_p - 1) & 1, abort_flag, P.status);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+          }
+          float part_lo = 0.f, part_hi = 0.f;
+          uint8_t* p_base = reinterpret_cast<uint8_t*>(sm.p);
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(t_s + ch * 32, r);
+            if (ch == 3) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+            }
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+            if (msk) apply_mask(v, j, ch);
+            uint32_t w[16];
+            float psum = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float t0 = fmaxf(fmaf(v[2 * e], P.c, -tau_c), 0.0f);
+              const float t1 = fmaxf(fmaf(v[2 * e + 1], P.c, -tau_c), 0.0f);
+              const float p0 = ALPHA2 ? t0 : t0 * t0;
+              const float p1 = ALPHA2 ? t1 : t1 * t1;
+              psum += p0 + p1;
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+              w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            if (ch < 2) part_lo += psum; else part_hi += psum;
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+              *reinterpret_cast<uint4*>(p_base + sw128_chunk_offset(rl, ch * 4 + qd)) =
+                  make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.p_full);
+          rowsum += part_lo + part_hi;
+          const uint32_t b_lo = __ballot_sync(0xffffffffu, row_ok && part_lo > 0.f);
+          const uint32_t b_hi = __ballot_sync(0xffffffffu, row_ok && part_hi > 0.f);
+          if (lane == 0) {
+            if (P.block == kTile) {
+              if (b_lo | b_hi) atomicOr(&sm.maskw[0][j >> 5], 1u << (j & 31));
+            } else {  // block 64: two mask rows per tile, two key blocks per tile
+              const int h = quad >> 1;
+              const int kb = 2 * j;
+              if (b_lo) atomicOr(&sm.maskw[h][kb >> 5], 1u << (kb & 31));
+              if (b_hi) atomicOr(&sm.maskw[h][(kb + 1) >> 5], 1u << ((kb + 1) & 31));
+            }
+          }
+        }
+      }
+
+      // ---------------- end of pass: solver step and the next tile list
+      auto build_list = [&](double thr_d) {
+        const float thr = row_ok ? __double2float_rd(thr_d) : INFINITY;
+        for (int t = 0; t < n; t += 4) {
+          float hv[4];
+          int jj[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            jj[u] = (t + u < n) ? static_cast<int>(sm.tiles[t + u]) : -1;
+            hv[u] = jj[u] >= 0 ? __half2float(P.tmax[tmax_index(bh, i, jj[u], P.tr, P.tc,
+                                                                 P.causal) + rl])
+                               : -INFINITY;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t b = __ballot_sync(0xffffffffu, hv[u] > thr);
+            if (lane == 0 && b != 0u && jj[u] >= 0)
+              atomicOr(&sm.flags[jj[u] >> 5], 1u << (jj[u] & 31));
+          }
+        }
+      };
+
+      if (kind == PASS_HIST) {
+        double tau_h = 0.0;
+        if (row_ok) {
+          if (fabsf(m_raw * P.cN) >= 2097152.0f) atomicOr(P.status, ST_RANGE);
+          // Reduced problem sum_b cnt_b [x_b - tau]_+^k = 1 with x_b = b / kNB
+          // (relative to the window base): scan candidate supports from the
+          // top bin down and take the first closed-form root that does not
+          // reach the next lower bin.
+          double C = 0.0, S1 = 0.0, S2 = 0.0, rel = 0.0;
+          bool found = false;
+#pragma unroll
+          for (int b = kNB; b >= 0; --b) {
+            const double cb = static_cast<double>(cnt[b]);
+            const double x = static_cast<double>(b) / kNB;
+            C += cb;
+            S1 += cb * x;
+            S2 += cb * x * x;
+            if (!found && C > 0.0) {
+              double cand;
+              bool valid = true;
+              if (ALPHA2) {
+                cand = (S1 - 1.0) / C;
+              } else {
+                const double disc = S1 * S1 - C * (S2 - 1.0);
+                valid = disc >= 0.0;
+                cand = (S1 - sqrt(fmax(disc, 0.0))) / C;
+              }
+              const double lower = (b == 0) ? -1e300 : static_cast<double>(b - 1) / kNB;
+              if (valid && cand >= lower) {
+                rel = cand;
+                found = true;
+              }
+            }
+          }
+          tau_h = static_cast<double>(gtop - kNB) / kNB + rel;
+          const double margin = 9.5367431640625e-07 * fmax(1.0, fabs(tau_h));  // 2^-20
+          const double m_s = static_cast<double>(m_raw) * P.c;
+          const double nb = ALPHA2 ? 1.0 / n_valid : 1.0 / sqrt(static_cast<double>(n_valid));
+          lo = tau_h - margin;
+          hi = fmin(tau_h + 1.0 / kNB + margin, m_s - nb + margin);
+          if (hi < lo) hi = lo;
+          tau_c = __double2float_rd(lo);
+          lo = tau_c;
+        }
+        iter = 0;
+        trace_store(0, static_cast<float>(tau_h));
+        build_list(lo);
+        epi_bar();
+        if (warp == 2) {
+          const int nn = compact_tiles(sm.flags, (ntc + 31) >> 5, sm.tiles);
+          if (lane == 0) {
+            sm.ctl_n = nn;
+            sm.ctl_kind = P.max_iter > 0 ? PASS_REFINE : PASS_PV;
+            atomicAdd(&P.counters[CNT_HIST_TILES], static_cast<unsigned long long>(n));
+          }
+        }
+      } else if (kind == PASS_REFINE) {
+        if (row_ok && !row_done) {
+          // f(tau) = sum_i [s_i - tau]_+^k - 1 at tau_c: F0 = sum t^k,
+          // F1 = sum t^(k-1), F2 = sum t^(k-2) (alpha = 1.5: k = 2; alpha = 2: k = 1).
+          const double f = F0 - 1.0;
+          if (f > 0.0) lo = fmax(lo, static_cast<double>(tau_c));
+          else if (f < 0.0) hi = fmin(hi, static_cast<double>(tau_c));
+          double tn = 0.5 * (lo + hi);
+          bool exact = (f == 0.0);
+          if (exact) {
+            tn = tau_c;
+          } else if (ALPHA2) {
+            // Newton: f is convex and piecewise linear, so the tangent root is a
+            // lower bound of tau*; it is tau* itself when no score of the
+            // current support is crossed (step < smallest positive gap).
+            if (F1 > 0.0) {
+              const double d = f / F1;
+              tn = tau_c + d;
+              lo = fmax(lo, tn);
+              exact = f > 0.0 && d < static_cast<double>(Tmin);
+            }
+          } else {
+            if (F1 > 0.0) {
+              // Newton lower bound (f convex).
+              lo = fmax(lo, tau_c + f / (2.0 * F1));
+              // On the current support f is the quadratic F2 d^2 - 2 F1 d + F0 - 1
+              // in d = tau - tau_c.  Its smaller root is tau* if it does not
+              // cross a support score, and an upper bound of tau* otherwise.
+              const double disc = F1 * F1 - F2 * f;
+              if (f > 0.0 && disc >= 0.0 && F2 > 0.0) {
+                const double dq = (F1 - sqrt(disc)) / F2;
+                if (dq <= static_cast<double>(Tmin)) {
+                  tn = tau_c + dq;
+                  exact = true;
+                } else {
+                  hi = fmin(hi, tau_c + dq);
+                }
+              }
+              if (!exact) {
+                const double fp = -2.0 * F1, fpp = 2.0 * F2;
+                tn = tau_c - 2.0 * f * fp / (2.0 * fp * fp - f * fpp);  // Halley
+              }
+            }
+          }
+          if (!exact && !(tn >= lo && tn <= hi)) tn = 0.5 * (lo + hi);  // bisection fallback
+          tau_c = static_cast<float>(tn);
+          if (exact) {
+            row_done = true;
+            lo = fmax(lo, static_cast<double>(__double2float_rd(tn)));
+          } else {
+            sm.not_converged = 1;
+          }
+        }
+        ++iter;
+        trace_store(iter, tau_c);
+        build_list(lo);
+        epi_bar();
+        if (warp == 2) {
+          const int nn = compact_tiles(sm.flags, (ntc + 31) >> 5, sm.tiles);
+          if (lane == 0) {
+            sm.ctl_n = nn;
+            sm.ctl_kind = (iter < P.max_iter && sm.not_converged) ? PASS_REFINE : PASS_PV;
+            sm.not_converged = 0;
+            atomicAdd(&P.counters[CNT_REFINE_TILES], static_cast<unsigned long long>(n));
+            atomicAdd(&P.counters[CNT_REFINE_PASSES], 1ull);
+          }
+        }
+      } else {  // PASS_PV: write O, tau, mask
+        if (ok && n > 0) {
+          ok = mbar_wait(&sm.o_full, 0, abort_flag, P.status);
+          ok = __all_sync(0xffffffffu, ok);
+        }
+        tc_fence_after();
+        __nv_bfloat16* orow = P.out + (static_cast<size_t>(bh) * P.N + row) * D;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t r[32];
+          if (ok && n > 0) {
+            tmem_ld32(t_lane + kColO + ch * 32, r);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          if (row_ok) {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const __nv_bfloat162 h2 =
+                  __floats2bfloat162_rn(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+              w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd)
+              dst[qd] = make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
+          }
+        }
+        if (row_ok) {
+          P.tau[static_cast<size_t>(bh) * P.N + row] = tau_c;
+          if (!(fabsf(rowsum - 1.0f) <= 1e-3f)) atomicOr(P.status, ST_NOT_CONVERGED);
+        }
+        for (int it = iter + 1; it <= P.max_iter; ++it) trace_store(it, tau_c);
+        tc_fence_before();
+        epi_bar();
+        const int spr = kTile / P.block;
+        const int et = threadIdx.x - 64;
+        for (int idx = et; idx < spr * P.mask_words; idx += kEpiThreads) {
+          const int h = idx / P.mask_words;
+          const int w = idx - h * P.mask_words;
+          const int mrow = i * spr + h;
+          if (mrow < P.mask_rows)
+            P.mask[(static_cast<size_t>(bh) * P.mask_rows + mrow) * P.mask_words + w] =
+                sm.maskw[h][w];
+        }
+        if (warp == 2 && lane == 0) {
+          sm.ctl_kind = PASS_DONE;
+          atomicAdd(&P.counters[CNT_PV_TILES], static_cast<unsigned long long>(n));
+        }
+      }
+    }
+  }
+
+  // ---------------- teardown: drain in-flight copies / MMAs after an abort,
+  // then release TMEM.
+  if (sm.abort_flag) {
+    if (warp == 0 && lane == 0) {
+      for (uint32_t s = 0; s < NS; ++s) {
+        if (kc > s) mbar_wait(&sm.k_full[s], ((kc - 1 - s) / NS) & 1, nullptr, nullptr);
+        if (vc > s) mbar_wait(&sm.v_full[s], ((vc - 1 - s) / NS) & 1, nullptr, nullptr);
+      }
+    }
+    if (warp == 1 && lane == 0) {
+      mma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, nullptr, nullptr);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace entmax

@@ -1,0 +1,182 @@
+/*
+ * entmax_attn.h -- C ABI of the B200 (sm_100a) alpha-entmax attention library.
+ *
+ * What is computed.  For every (batch b, head h) and query row r:
+ *     z_rc = q_r . k_c / sqrt(D)            (causal: only keys c <= r)
+ *     s_rc = (alpha - 1) * z_rc
+ *     p_rc = [ s_rc - tau_r ]_+ ^ (1/(alpha-1)),  tau_r chosen so sum_c p_rc = 1
+ *     O_r  = sum_c p_rc v_c
+ * alpha-entmax is the sparse, differentiable softmax replacement that the
+ * AdaSplash-2 summaries ("AdaSplash-2: Faster Differentiable Sparse
+ * Attention", zh/it/ja/es pages, section 1) build on; tau is the normaliser
+ * they liken to log-sum-exp.  tau is reported in s-units (the units of s
+ * above, i.e. (alpha-1) * z).
+ *
+ * How (zh §2.1-2.3, it §2A-2C, ja §2.1-2.3, es §2A-2C): one streaming pass
+ * over the key blocks builds an on-chip histogram of the scores per query row
+ * and solves the reduced problem for a lower bound tau_h of tau; one or two
+ * safeguarded Halley (alpha = 1.5) or Newton (alpha = 2) steps refine it; a
+ * bit-packed block mask (32 blocks per uint32) records the non-zero blocks and
+ * P.V, dQ, dK and dV visit only those blocks.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no memory: scratch space is the caller's `workspace`.
+ *   - q, k, v, out, dout, dq, dk, dv: contiguous [B][H][N][D], element type
+ *     `dtype` (ENTMAX_DTYPE_BF16 or ENTMAX_DTYPE_FP32), 16-byte aligned.
+ *   - tau: float32 [B][H][N].  mask: uint32 [B][H][Tb][W] with
+ *     Tb = ceil(N / block) row blocks and W = entmax_attn_mask_words(N, block)
+ *     words per row block; bit (j % 32) of word j / 32 is key block j (least
+ *     significant bit = lowest block index).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; a return of ENTMAX_OK means the work
+ *     was enqueued, not that it finished.
+ *   - Arguments are validated before anything is enqueued; on an error return
+ *     nothing has been launched and no output was touched.
+ *   - Conditions found on the device (a row whose probabilities do not sum to
+ *     1 within 1e-3, a bounded wait that timed out, an out-of-range score) are
+ *     OR-ed into a status word at the start of the workspace; read it with
+ *     entmax_attn_status().  Kernels never trap.
+ *   - Supported: D in {64, 128}; block in {64, 128}; alpha in {1.5, 2.0};
+ *     1 <= N <= ENTMAX_MAX_N; dtype bf16 (tensor-core path) or fp32.
+ */
+#ifndef ENTMAX_ATTN_H
+#define ENTMAX_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define ENTMAX_OK             0
+#define ENTMAX_E_NULL        -1  /* a required pointer is NULL                     */
+#define ENTMAX_E_ALIGN       -2  /* a tensor pointer is not 16-byte aligned         */
+#define ENTMAX_E_SHAPE       -3  /* B, H or N out of range                          */
+#define ENTMAX_E_UNSUPPORTED -4  /* D, dtype or block not supported                 */
+#define ENTMAX_E_ALPHA       -5  /* alpha not supported                             */
+#define ENTMAX_E_WORKSPACE   -6  /* workspace smaller than entmax_attn_workspace_size */
+#define ENTMAX_E_CUDA        -7  /* a CUDA call failed (launch, tensor-map encode)  */
+#define ENTMAX_E_MAXITER     -8  /* max_iter outside [0, ENTMAX_MAX_ITER]            */
+
+/* element types */
+#define ENTMAX_DTYPE_BF16 0
+#define ENTMAX_DTYPE_FP32 1
+
+/* device status bits (entmax_attn_status) */
+#define ENTMAX_ST_NOT_CONVERGED 1u /* some row's sum of p is off 1 by more than 1e-3 */
+#define ENTMAX_ST_TIMEOUT       2u /* a bounded wait gave up; outputs are not valid   */
+#define ENTMAX_ST_RANGE         4u /* |s| * 8 reached 2^21 somewhere: histogram inexact */
+
+#define ENTMAX_MAX_N    262144
+#define ENTMAX_MAX_ITER 8
+
+/*
+ * Number of uint32 words per row block of the block mask: ceil(ceil(N/block)/32).
+ * Returns a negative error code for unsupported N or block.
+ */
+int entmax_attn_mask_words(int N, int block);
+
+/*
+ * Bytes of device workspace that entmax_attn_fwd and entmax_attn_bwd need for
+ * this problem (the same buffer serves both).  It holds the status word and
+ * work counters, the per-(row, key tile) score maxima of the histogram pass
+ * (fp16, rounded up), the tile-granularity mask and its transpose, the per-row
+ * delta of the backward and the backward's fp16 copies of q, k, v and dout.
+ * Returns 0 for unsupported arguments.
+ */
+size_t entmax_attn_workspace_size(int B, int H, int N, int D, int block, int causal);
+
+/*
+ * Forward pass.  AdaSplash-2 zh §2.1 (histogram initialisation), §2.2 (hybrid
+ * solver, one or two iterations), §2.3 (bit-packed block mask, zero-block
+ * skipping); it §2A-2C; ja §2.1-2.3; es §2A-2C.
+ *
+ *   q, k, v      in   [B][H][N][D], dtype.
+ *   alpha        in   1.5 (Halley steps) or 2.0 (Newton steps).
+ *   causal       in   nonzero: key c is visible to query r iff c <= r.
+ *   block        in   block size of the mask (64 or 128), rows and keys alike.
+ *   max_iter     in   at most this many refinement passes after the histogram
+ *                     bound (0..8).  A row stops once its threshold is
+ *                     certified exact -- the step did not cross any score of
+ *                     the current support, so the closed-form root on that
+ *                     support is tau* -- and a 128-row tile stops once all of
+ *                     its rows have; the summaries report 1, at most 2,
+ *                     iterations (zh §2.2), 4 is a safe cap.
+ *   out          out  [B][H][N][D], dtype.
+ *   tau          out  float32 [B][H][N], s-units.
+ *   mask         out  uint32 [B][H][ceil(N/block)][W], bit set iff the block
+ *                     holds a non-zero probability (at the final tau).
+ *   tau_trace    out  optional (NULL = off): float32 [max_iter+1][B][H][N];
+ *                     entry 0 is the histogram bound tau_h, entry i the
+ *                     threshold after refinement step i.
+ *   workspace    in/out  device buffer of >= entmax_attn_workspace_size() bytes,
+ *                     256-byte aligned; its status word is cleared here.
+ */
+int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int D,
+                    int dtype, float alpha, int causal, int block, int max_iter, void* out,
+                    float* tau, uint32_t* mask, float* tau_trace, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass over the forward's mask (zh §2.3 and ja §2.3: zero blocks are
+ * skipped in the backward as well; ja §2.3: local accumulators instead of
+ * atomics).  With g = p^(2-alpha) on the support:
+ *     dP = dO V^T,  delta_r = sum_c g dP / sum_c g,  dZ = g (dP - delta)
+ *     dQ = dZ K / sqrt(D),  dK = dZ^T Q / sqrt(D),  dV = P^T dO
+ *
+ *   q, k, v, dout  in  [B][H][N][D], dtype.
+ *   tau, mask      in  exactly as written by entmax_attn_fwd for these inputs.
+ *   alpha, causal, block   as given to entmax_attn_fwd.
+ *   dq, dk, dv     out [B][H][N][D], dtype (fully overwritten).
+ *   workspace      in/out  the same size rule as for the forward; status bits
+ *                  are OR-ed into the existing status word.
+ * The backward's MMAs run on exact fp16 copies of the bf16 inputs, so that
+ * the operands rounded on chip (P and dS) keep 11 significant bits; an input
+ * of magnitude above 65504 (outside fp16) raises ENTMAX_ST_RANGE.
+ */
+int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                    const float* tau, const uint32_t* mask, int B, int H, int N, int D,
+                    int dtype, float alpha, int causal, int block, void* dq, void* dk, void* dv,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream` and copies the device status word (ENTMAX_ST_* bits)
+ * of `workspace` to *status.  Returns ENTMAX_E_CUDA if the stream reported an
+ * error (e.g. from an earlier launch).
+ */
+int entmax_attn_status(const void* workspace, void* stream, uint32_t* status);
+
+/*
+ * Diagnostics: copies the first n (1..8) work counters of `workspace` to
+ * counters[] after synchronising `stream`.  [0] key tiles visited by the
+ * forward's histogram pass, [1] by its refinement passes, [2] by its P.V pass,
+ * [3] refinement passes summed over 128-row tiles, [4] active key tiles per
+ * pass of the backward row kernel, [5] active query tiles of the backward
+ * column kernel (tiles are 128 x 128).  Cleared by entmax_attn_fwd ([0]-[3])
+ * and entmax_attn_bwd ([4]-[5]).
+ */
+int entmax_attn_counters(const void* workspace, void* stream, unsigned long long* counters, int n);
+
+/*
+ * Profiling aid, off by default and per calling thread.  entmax_attn_profile(1)
+ * makes the thread's later fwd/bwd calls record CUDA events on their stream
+ * around each kernel (it creates the events once; no memory is allocated);
+ * entmax_attn_profile(0) stops recording.  entmax_attn_profile_read() waits for
+ * the last recorded events and writes up to 5 durations in ms: [0] forward
+ * kernel, [1] backward fp16 operand copies, [2] backward tile-mask preparation,
+ * [3] backward row kernel (delta, dQ), [4] backward column kernel (dK, dV).
+ */
+int entmax_attn_profile(int enable);
+int entmax_attn_profile_read(float* ms, int n);
+
+/* Static, human-readable text for a return code. */
+const char* entmax_attn_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENTMAX_ATTN_H */

@@ -1,0 +1,107 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function that include/entmax_attn.h declares, and rejects invalid
+arguments before touching any device state.
+
+Every call below fails validation before any CUDA call is made, so the fake
+(but aligned, non-null) pointers are never dereferenced.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import differentiable_sparse_attention_b200 as dsa
+from differentiable_sparse_attention_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "entmax_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return dsa._lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(entmax_attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert set(names) == set(dsa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert getattr(lib, name) is not None
+
+
+FAKE = ctypes.c_void_p(1 << 20)          # 256-byte aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+
+
+def fwd(lib, *, q=FAKE, B=1, H=1, N=256, D=64, dtype=0, alpha=1.5, causal=1, block=128,
+        max_iter=2, out=FAKE, ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.entmax_attn_workspace_size(B, H, N, D, block, causal) if N > 0 else 0
+    return lib.entmax_attn_fwd(q, FAKE, FAKE, B, H, N, D, dtype, alpha, causal, block, max_iter,
+                               out, FAKE, FAKE, None, ws, ws_bytes, None)
+
+
+def test_forward_argument_validation(lib):
+    assert fwd(lib, q=None) == dsa.E_NULL
+    assert fwd(lib, out=None) == dsa.E_NULL
+    assert fwd(lib, ws=None) == dsa.E_NULL
+    assert fwd(lib, N=0) == dsa.E_SHAPE
+    assert fwd(lib, N=262145) == dsa.E_SHAPE
+    assert fwd(lib, B=0) == dsa.E_SHAPE
+    assert fwd(lib, D=96) == dsa.E_UNSUPPORTED
+    assert fwd(lib, block=32) == dsa.E_UNSUPPORTED
+    assert fwd(lib, dtype=7) == dsa.E_UNSUPPORTED
+    assert fwd(lib, alpha=1.0) == dsa.E_ALPHA
+    assert fwd(lib, alpha=1.7) == dsa.E_ALPHA
+    assert fwd(lib, max_iter=-1) == dsa.E_MAXITER
+    assert fwd(lib, max_iter=9) == dsa.E_MAXITER
+    assert fwd(lib, q=MISALIGNED) == dsa.E_ALIGN
+    assert fwd(lib, ws_bytes=1) == dsa.E_WORKSPACE
+
+
+def test_backward_argument_validation(lib):
+    def bwd(q=FAKE, D=64, block=128, alpha=1.5, ws_bytes=None, dq=FAKE):
+        if ws_bytes is None:
+            ws_bytes = lib.entmax_attn_workspace_size(1, 1, 256, 64, 128, 1)
+        return lib.entmax_attn_bwd(q, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 256, D, 0, alpha, 1,
+                                   block, dq, FAKE, FAKE, FAKE, ws_bytes, None)
+    assert bwd(q=None) == dsa.E_NULL
+    assert bwd(dq=None) == dsa.E_NULL
+    assert bwd(D=32) == dsa.E_UNSUPPORTED
+    assert bwd(alpha=3.0) == dsa.E_ALPHA
+    assert bwd(q=MISALIGNED) == dsa.E_ALIGN
+    assert bwd(ws_bytes=0) == dsa.E_WORKSPACE
+
+
+def test_sizes(lib):
+    assert dsa.mask_words(256, 64) == 1
+    assert dsa.mask_words(4096, 128) == 1
+    assert dsa.mask_words(131072, 128) == 32
+    assert dsa.mask_words(300, 64) == 1
+    assert lib.entmax_attn_mask_words(0, 128) == dsa.E_SHAPE
+    assert lib.entmax_attn_mask_words(256, 96) == dsa.E_UNSUPPORTED
+    small = dsa.workspace_size(1, 1, 256, 64, 128, True)
+    big = dsa.workspace_size(1, 1, 4096, 64, 128, True)
+    assert 0 < small < big
+    # causal keeps only the lower triangle of tile maxima
+    assert dsa.workspace_size(2, 16, 4096, 64, 128, True) < dsa.workspace_size(2, 16, 4096, 64, 128, False)
+    assert dsa.workspace_size(1, 1, 0, 64, 128, True) == 0
+
+
+def test_error_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -99):
+        s = dsa.error_string(code)
+        assert isinstance(s, str) and s

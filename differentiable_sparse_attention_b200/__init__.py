@@ -19,13 +19,15 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libentmax_attn.so")
 
 OK = 0
-E_NULL, E_ALIGN, E_SHAPE, E_UNSUPPORTED, E_ALPHA, E_WORKSPACE, E_CUDA, E_MAXITER = (
-    -1, -2, -3, -4, -5, -6, -7, -8)
+E_NULL, E_ALIGN, E_SHAPE, E_UNSUPPORTED, E_ALPHA, E_WORKSPACE, E_CUDA, E_MAXITER, E_SCRATCH = (
+    -1, -2, -3, -4, -5, -6, -7, -8, -9)
+NOALLOC_SCRATCH_BYTES = 8 << 20
 ST_NOT_CONVERGED, ST_TIMEOUT, ST_RANGE = 1, 2, 4
 DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
 EXPORTED = ("entmax_attn_mask_words", "entmax_attn_workspace_size", "entmax_attn_fwd",
             "entmax_attn_bwd", "entmax_attn_status", "entmax_attn_counters",
-            "entmax_attn_profile", "entmax_attn_profile_read", "entmax_attn_error_string")
+            "entmax_attn_profile", "entmax_attn_profile_read", "entmax_attn_error_string",
+            "entmax_attn_fwd_noalloc")
 COUNTER_NAMES = ("fwd_hist_tiles", "fwd_refine_tiles", "fwd_pv_tiles", "fwd_refine_passes",
                  "bwd_row_tiles", "bwd_col_tiles")
 PHASE_NAMES = ("fwd", "bwd_fp16_copies", "bwd_tile_masks", "bwd_row", "bwd_col")
@@ -68,6 +70,9 @@ def _lib():
     lib.entmax_attn_profile.restype = c_int
     lib.entmax_attn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), c_int]
     lib.entmax_attn_profile_read.restype = c_int
+    lib.entmax_attn_fwd_noalloc.argtypes = ([vp, vp, vp] + [c_int] * 5
+                                            + [c_float, c_int, c_int, c_int] + [vp] * 4)
+    lib.entmax_attn_fwd_noalloc.restype = c_int
     lib.entmax_attn_error_string.argtypes = [c_int]
     lib.entmax_attn_error_string.restype = ctypes.c_char_p
     _lib_handle = lib

@@ -160,6 +160,30 @@ int launch_bwd_col(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
 }
 
+// ------------------------------------------------------------ fixed scratch
+// Scratch for entmax_attn_fwd_noalloc: status word and counters (first 256
+// bytes) followed by the forward's per-(row, key tile) maxima.  It is part of
+// the loaded module, so each GPU that loads this library holds these 8 MiB
+// until the process exits.  Every call of entmax_attn_fwd_noalloc on a device
+// reuses the same bytes.
+constexpr size_t kNoAllocScratchBytes = 8u << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, resolved once per device (in host code
+// the symbol itself is only a host-side handle, not a device address).
+void* noalloc_scratch_ptr(int device) {
+  static std::mutex mu;
+  static void* ptrs[256] = {};
+  if (device < 0 || device >= 256) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[device] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    ptrs[device] = p;
+  }
+  return ptrs[device];
+}
+
 }  // namespace
 
 // ============================================================== C ABI
@@ -233,6 +257,63 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
   }
   prof_mark(EV_FWD1, st);
   return rc;
+}
+
+int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, int H, int N,
+                            int D, int dtype, float alpha, int causal, int block, int max_iter,
+                            void* out, float* tau, uint32_t* mask, void* stream) {
+  if (!q || !k || !v || !out || !tau || !mask) return ENTMAX_E_NULL;
+  int rc = check_common(B, H, N, D, dtype, alpha, block);
+  if (rc != ENTMAX_OK) return rc;
+  if (max_iter < 0 || max_iter > ENTMAX_MAX_ITER) return ENTMAX_E_MAXITER;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(tau) ||
+      !aligned16(mask))
+    return ENTMAX_E_ALIGN;
+  // Only the forward's part of the workspace layout is needed: the first 256
+  // bytes and the tile maxima that follow them.
+  const WsLayout L = ws_layout(B, H, N, D, causal ? 1 : 0);
+  if (L.tilemask > kNoAllocScratchBytes) return ENTMAX_E_SCRATCH;
+
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return ENTMAX_E_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(noalloc_scratch_ptr(device));
+  if (ws == nullptr) return ENTMAX_E_CUDA;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
+    return ENTMAX_E_CUDA;
+  // status word and counters must start at zero; the tile maxima are written
+  // before they are read by each CTA.
+  if (cudaMemsetAsync(ws + L.status, 0, 8 + CNT_COUNT * sizeof(unsigned long long), st) != cudaSuccess)
+    return ENTMAX_E_CUDA;
+
+  FwdParams p{};
+  p.BH = BH;
+  p.N = N;
+  p.tr = (N + kTile - 1) / kTile;
+  p.tc = p.tr;
+  p.causal = causal ? 1 : 0;
+  p.block = block;
+  p.mask_rows = (N + block - 1) / block;
+  p.mask_words = (p.mask_rows + 31) / 32;
+  p.max_iter = max_iter;
+  p.c = (alpha - 1.0f) / std::sqrt(static_cast<float>(D));
+  p.cN = p.c * static_cast<float>(kNB);
+  p.slim = 2097152.0f / p.cN;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.tau = tau;
+  p.mask = mask;
+  p.tau_trace = nullptr;
+  p.tmax = reinterpret_cast<__half*>(ws + L.tmax);
+  p.status = reinterpret_cast<uint32_t*>(ws + L.status);
+  p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
+
+  const bool a2 = alpha == 2.0f;
+  if (D == 64)
+    return a2 ? launch_fwd<64, 3, true>(mq, mk, mv, p, st) : launch_fwd<64, 3, false>(mq, mk, mv, p, st);
+  return a2 ? launch_fwd<128, 2, true>(mq, mk, mv, p, st) : launch_fwd<128, 2, false>(mq, mk, mv, p, st);
 }
 
 int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
@@ -388,6 +469,8 @@ const char* entmax_attn_error_string(int code) {
     case ENTMAX_E_WORKSPACE: return "workspace smaller than entmax_attn_workspace_size()";
     case ENTMAX_E_CUDA: return "a CUDA call failed";
     case ENTMAX_E_MAXITER: return "max_iter out of range";
+    case ENTMAX_E_SCRATCH:
+      return "problem needs more scratch than entmax_attn_fwd_noalloc's fixed 8 MiB";
     default: return "unknown error code";
   }
 }

@@ -60,6 +60,8 @@ extern "C" {
 #define ENTMAX_E_WORKSPACE   -6  /* workspace smaller than entmax_attn_workspace_size */
 #define ENTMAX_E_CUDA        -7  /* a CUDA call failed (launch, tensor-map encode)  */
 #define ENTMAX_E_MAXITER     -8  /* max_iter outside [0, ENTMAX_MAX_ITER]            */
+#define ENTMAX_E_SCRATCH     -9  /* entmax_attn_fwd_noalloc: problem needs more than
+                                    ENTMAX_NOALLOC_SCRATCH_BYTES of scratch          */
 
 /* element types */
 #define ENTMAX_DTYPE_BF16 0
@@ -72,6 +74,7 @@ extern "C" {
 
 #define ENTMAX_MAX_N    262144
 #define ENTMAX_MAX_ITER 8
+#define ENTMAX_NOALLOC_SCRATCH_BYTES (8u << 20)
 
 /*
  * Number of uint32 words per row block of the block mask: ceil(ceil(N/block)/32).
@@ -119,6 +122,37 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
                     int dtype, float alpha, int causal, int block, int max_iter, void* out,
                     float* tau, uint32_t* mask, float* tau_trace, void* workspace,
                     size_t workspace_bytes, void* stream);
+
+/*
+ * Forward pass without a workspace argument, for callers that cannot obtain
+ * device memory at call time: code that runs where cudaMalloc is unavailable
+ * or forbidden (inside a host callback or another library's critical section,
+ * under an allocator that must not grow, or in a plain C program that owns no
+ * allocator).  The paper has no counterpart to this entry point; it exists
+ * only for such callers.
+ *
+ * It computes exactly what entmax_attn_fwd computes (same kernel, same
+ * arguments and outputs, no tau_trace), but its scratch -- status word, work
+ * counters and the histogram pass's tile maxima -- lives in one fixed device
+ * array of ENTMAX_NOALLOC_SCRATCH_BYTES (8 MiB) that is part of this library:
+ * every GPU that loads the library holds those 8 MiB until the process exits.
+ * The call allocates nothing and calls no allocating routine.
+ *   - Problems whose scratch exceeds the 8 MiB return ENTMAX_E_SCRATCH and
+ *     launch nothing (causal: 256 + B*H*T*(T+1)/2*256 bytes, T = ceil(N/128);
+ *     e.g. B*H = 32 at N = 4096 needs 4.3 MB).
+ *   - The array's device address is looked up once per device, on the first
+ *     call made while that device is current; make that first call before any
+ *     stream capture on the device.
+ *   - All calls on a device share the one array, which keeps the previous
+ *     call's contents; the call clears the parts that must start at zero.
+ *     Calls whose kernels may overlap on the GPU (other streams, other host
+ *     threads) race on the array: serialise them.
+ *   - The status word stays in the library's array and is not reported; use
+ *     entmax_attn_fwd when the device status is needed.
+ */
+int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, int H, int N,
+                            int D, int dtype, float alpha, int causal, int block, int max_iter,
+                            void* out, float* tau, uint32_t* mask, void* stream);
 
 /*
  * Backward pass over the forward's mask (zh §2.3 and ja §2.3: zero blocks are

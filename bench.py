@@ -105,10 +105,16 @@ class ClockSampler:
                 stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return self
+        # wait (up to 3 s) for the first sample so the timed region is covered
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
         return self
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(0.25)  # one more sample at the end of the timed region
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -400,8 +406,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override H (small cases for profiler captures)")
     args = ap.parse_args()
     points = workload_points(args.workload)
+    if args.heads:
+        points = [p.with_(H=args.heads) for p in points]
     args.workload_desc = (f"{args.workload}: " + ", ".join(
         f"B={p.B} H={p.H} N={p.N} D={p.D} alpha={p.alpha} t={p.temperature}"
         + (f" planted={p.planted_blocks}" if p.planted_blocks else "") for p in points)

@@ -29,7 +29,7 @@ EXPORTED = ("entmax_attn_mask_words", "entmax_attn_workspace_size", "entmax_attn
             "entmax_attn_profile", "entmax_attn_profile_read", "entmax_attn_error_string",
             "entmax_attn_fwd_noalloc")
 COUNTER_NAMES = ("fwd_hist_tiles", "fwd_refine_tiles", "fwd_pv_tiles", "fwd_refine_passes",
-                 "bwd_row_tiles", "bwd_col_tiles")
+                 "bwd_row_tiles", "bwd_col_tiles", "fwd_cand_overflow_tiles")
 PHASE_NAMES = ("fwd", "bwd_fp16_copies", "bwd_tile_masks", "bwd_row", "bwd_col")
 
 _lib_handle = None

@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
         }
         const bool msk = (P.causal && j == i) || ((j + 1) * kTile > P.N);
-        float a_gdp = 0.f, a_g = 0.f;
+        float a_gdp[4] = {0.f, 0.f, 0.f, 0.f}, a_g[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t rs[32], rp[32];
@@ -360,8 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (pass == 0) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              a_gdp = fmaf(gg[e], __uint_as_float(rp[e]), a_gdp);
-              a_g += gg[e];
+              a_gdp[e & 3] = fmaf(gg[e], __uint_as_float(rp[e]), a_gdp[e & 3]);
+              a_g[e & 3] += gg[e];
             }
           } else {
             uint32_t w[16];
@@ -379,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (pass == 0) {
-          gdp += a_gdp;
-          gsum += a_g;
+          gdp += (a_gdp[0] + a_gdp[1]) + (a_gdp[2] + a_gdp[3]);
+          gsum += (a_g[0] + a_g[1]) + (a_g[2] + a_g[3]);
         } else {
           fence_proxy_async_smem();
           __syncwarp();

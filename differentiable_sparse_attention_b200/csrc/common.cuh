@@ -21,7 +21,7 @@ constexpr int kNB = 8;                       // histogram bins per unit of s
 constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23
 constexpr uint32_t kMagicBits = 0x4B400000u; // bit pattern of kMagic
 
-enum PassKind : int { PASS_HIST = 0, PASS_REFINE = 1, PASS_PV = 2, PASS_DONE = 3 };
+enum PassKind : int { PASS_HIST = 0, PASS_REFINE = 1, PASS_PV = 2, PASS_DONE = 3, PASS_COLLECT = 4 };
 
 // Work counters kept in the workspace right after the status word (uint64 each).
 enum Counter : int {
@@ -31,8 +31,10 @@ enum Counter : int {
   CNT_REFINE_PASSES = 3, // forward: refinement passes, summed over 128-row tiles
   CNT_ROW_TILES = 4,     // backward: key tiles per pass of the row kernel
   CNT_COL_TILES = 5,     // backward: query tiles visited by the column kernel
+  CNT_CAND_OVERFLOW = 6, // forward: 128-row tiles whose candidate lists overflowed
   CNT_COUNT = 8
 };
+
 
 // Named barrier over the four epilogue warps only (id 1; id 0 is __syncthreads).
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -63,6 +65,20 @@ __device__ __forceinline__ uint32_t sw128_chunk_offset(int row, int chunk16) {
   const int slab = chunk16 >> 3;
   const int c = chunk16 & 7;
   return static_cast<uint32_t>(slab * kSlabBytes + row * 128 + ((c ^ (row & 7)) << 4));
+}
+
+// Maximum of 32 values as a 5-level tree (a linear chain would serialise 31
+// dependent max operations in the epilogue).
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+  float m[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) m[e] = fmaxf(v[e], v[e + 16]);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int e = 0; e < w; ++e) m[e] = fmaxf(m[e], m[e + w]);
+  }
+  return m[0];
 }
 
 // Warp-parallel compaction of the set bits of flags[0, nwords) into a sorted

@@ -245,6 +245,7 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
   p.mask = mask;
   p.tau_trace = tau_trace;
   p.tmax = reinterpret_cast<__half*>(ws + L.tmax);
+  p.inv_c = std::nextafter(1.0f / p.c, INFINITY) * (1.0f + 1e-6f);
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
 
@@ -307,6 +308,7 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, 
   p.mask = mask;
   p.tau_trace = nullptr;
   p.tmax = reinterpret_cast<__half*>(ws + L.tmax);
+  p.inv_c = std::nextafter(1.0f / p.c, INFINITY) * (1.0f + 1e-6f);
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
 

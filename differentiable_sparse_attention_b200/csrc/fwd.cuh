@@ -21,6 +21,8 @@
 //           (32 blocks per uint32 word, zh §2.3) of blocks holding a p > 0.
 #pragma once
 
+#include <cstddef>
+
 #include "common.cuh"
 
 namespace entmax {
@@ -39,9 +41,117 @@ struct FwdParams {
   uint32_t* mask;
   float* tau_trace;          // nullable, [max_iter + 1][BH][N]
   __half* tmax;              // workspace: per-(row, key tile) maxima of s, rounded up
+  float inv_c;               // 1 / c rounded up
   uint32_t* status;          // workspace word 0
   unsigned long long* counters;  // workspace, CNT_* work counters
 };
+
+// tau_h: exact root of the reduced histogram problem.  cnt[b] counts the scores
+// of grid bin gtop - kNB + b (bin width 1/kNB in s-units, lower edge as the
+// representative); with x_b = b / kNB the problem is
+// sum_b cnt_b [x_b - tau]_+^k = 1 relative to the window base.  Candidate
+// supports are scanned from the top bin down; the first closed-form root that
+// does not reach the next lower bin is the root (zh §2.1: the n scores become
+// a sum over the bins).  Returns tau_h in s-units.
+template <bool ALPHA2, typename R = double>
+__device__ __forceinline__ R hist_threshold(const uint32_t (&cnt)[kNB + 1], int gtop) {
+  // Scanning from the top bin, the first support {b..kNB} whose reduced
+  // function is still >= 0 at the next lower edge x_(b-1) holds the root (it
+  // decreases, and at its own lower edge x_b it is already < 0):
+  // C x^2 - 2 S1 x + S2 - 1 >= 0 for alpha = 1.5, S1 - C x - 1 >= 0 for
+  // alpha = 2.  Only the selected support's closed-form root is evaluated.
+  R C = 0, S1 = 0, S2 = 0;
+  R Cs = 0, S1s = 0, S2s = 0;
+  bool found = false;
+#pragma unroll
+  for (int b = kNB; b >= 0; --b) {
+    const R cb = static_cast<R>(cnt[b]);
+    const R x = static_cast<R>(b) / kNB;
+    C += cb;
+    S1 += cb * x;
+    S2 += cb * x * x;
+    if (!found && C > R(0)) {
+      bool holds = true;
+      if (b > 0) {
+        const R xl = static_cast<R>(b - 1) / kNB;
+        holds = ALPHA2 ? (S1 - C * xl - R(1)) >= R(0)
+                       : (C * xl * xl - R(2) * S1 * xl + S2 - R(1)) >= R(0);
+      }
+      if (holds) {
+        found = true;
+        Cs = C;
+        S1s = S1;
+        S2s = S2;
+      }
+    }
+  }
+  R rel;
+  if (ALPHA2) {
+    rel = (S1s - R(1)) / Cs;
+  } else {
+    const R disc = S1s * S1s - Cs * (S2s - R(1));
+    rel = (S1s - sqrt(disc > R(0) ? disc : R(0))) / Cs;
+  }
+  return static_cast<R>(gtop - kNB) / kNB + rel;
+}
+
+// Safety margin below tau_h that absorbs the rounding of s and tau (2^-20 |tau|).
+__device__ __forceinline__ double hist_margin(double tau_h) {
+  return 9.5367431640625e-07 * fmax(1.0, fabs(tau_h));
+}
+
+// One safeguarded refinement step from tau_c (zh §2.2, it §2B, ja §2.2, es §2B).
+// F0 = sum t^k, F1 = sum t^(k-1), F2 = sum t^(k-2) over the support S = {t > 0},
+// t = s - tau_c (alpha = 1.5: k = 2; alpha = 2: k = 1); tmin / tneg are the
+// smallest positive and the largest non-positive t seen; every score left out
+// of the sums lies at or below l_drop.  The bracket [lo, hi] is updated from
+// the sign of f, then r, the root of f restricted to S (linear for alpha = 2,
+// the smaller root of the quadratic F2 d^2 - 2 F1 d + f in d = tau - tau_c for
+// alpha = 1.5), is tau* when no score lies between tau_c and r -- the support
+// does not change on the way -- and bounds tau* otherwise: from the right it is
+// a lower bound, from the left a lower bound for alpha = 2 (f is convex) and an
+// upper bound for alpha = 1.5 ([x]_+^2 <= x^2).  Without that certificate the
+// next point is the Newton (alpha = 2) or Halley (alpha = 1.5) step, replaced
+// by bisection when it leaves the bracket.  Returns true when tau_c is exact.
+template <bool ALPHA2>
+__device__ __forceinline__ bool solver_step(double F0, double F1, double F2, float tmin,
+                                            float tneg, double l_drop, float& tau_c, double& lo,
+                                            double& hi) {
+  const double f = F0 - 1.0;
+  if (f > 0.0) lo = fmax(lo, static_cast<double>(tau_c));
+  else if (f < 0.0) hi = fmin(hi, static_cast<double>(tau_c));
+  bool exact = (f == 0.0);
+  double tn = tau_c;
+  double r = NAN;
+  if (!exact && F1 > 0.0) {
+    if (ALPHA2) {
+      r = tau_c + f / F1;
+    } else {
+      const double disc = F1 * F1 - F2 * f;
+      if (disc >= 0.0 && F2 > 0.0) r = tau_c + (F1 - sqrt(disc)) / F2;
+    }
+    if (!isnan(r)) {
+      const double d = r - tau_c;
+      exact = f > 0.0 ? d <= static_cast<double>(tmin)
+                      : (d >= static_cast<double>(tneg) && r >= l_drop);
+      if (exact) tn = r;
+      else if (ALPHA2 || f < 0.0) lo = fmax(lo, r);
+      else hi = fmin(hi, r);
+    }
+  }
+  if (!exact) {
+    if (ALPHA2) {
+      tn = r;                                                    // Newton step
+    } else {
+      const double fp = -2.0 * F1, fpp = 2.0 * F2;
+      tn = tau_c - 2.0 * f * fp / (2.0 * fp * fp - f * fpp);     // Halley step
+    }
+    if (!(tn >= lo && tn <= hi)) tn = 0.5 * (lo + hi);           // bisection fallback
+  }
+  tau_c = static_cast<float>(tn);
+  if (exact) lo = fmax(lo, static_cast<double>(__double2float_rd(tn)));
+  return exact;
+}
 
 template <int D, int NS>
 struct FwdSmem {
@@ -58,10 +168,22 @@ struct FwdSmem {
   int abort_flag;
   int ctl_kind, ctl_n, ctl_iter;
   int not_converged;
+  int cand_overflow;
   uint32_t flags[kMaxTiles / 32];
   uint32_t maskw[2][kMaxMaskWords];
   uint16_t tiles[kMaxTiles];
 };
+
+// Candidate scores live in the V ring and the P tile, which stay idle until
+// the P.V pass: slot-major [cap][128 rows] floats (thread r uses column r, so
+// appends and reads are free of bank conflicts).  A row compacts its list at
+// most kMaxPrunes times; after that its list is rebuilt by a COLLECT pass.
+constexpr int kMaxPrunes = 2;
+
+template <int D, int NS>
+__host__ __device__ constexpr int fwd_cand_cap() {
+  return (NS * kTile * D * 2 + kTile * kTile * 2) / (4 * kTile);
+}
 
 template <int D, int NS>
 constexpr size_t fwd_smem_bytes() {
@@ -111,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     sm.not_converged = 0;
+    sm.cand_overflow = 0;
     sm.ctl_kind = PASS_HIST;
     sm.ctl_n = ntc;
     sm.ctl_iter = 0;
@@ -153,14 +276,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int b = 0; b <= kNB; ++b) cnt[b] = 0u;
   float vclamp = -P.slim;                  // scores are clamped to >= vclamp before binning
   uint32_t cbase = 0u;
+  // Candidate scores of this row: every q.k above acc_raw, which only grows and
+  // always stays at or below a lower bound of tau* (c * acc_raw <= tau*): the
+  // running max minus 1/c, raised to a partial-histogram tau_h when the list
+  // fills up and is pruned.  Scores left out are never in the support.
+  constexpr int kCap = fwd_cand_cap<D, NS>();
+  using Smem = FwdSmem<D, NS>;
+  static_assert(offsetof(Smem, p) == offsetof(Smem, v) + NS * kTile * D * 2,
+                "candidates need the V ring and the P tile to be adjacent");
+  float* my_cand = reinterpret_cast<float*>(&sm.v[0][0]) + rl;   // slot a at my_cand[a * 128]
+  int ncand = 0;
+  float acc_raw = -INFINITY;
+  bool cand_over = false;
+  int prunes = 0;                          // list compactions so far (at most kMaxPrunes)
+  bool collect = false;                    // list rebuilt by a COLLECT pass above lo
   double lo = 0.0, hi = 0.0;               // bracket of tau*
+  double l_drop = -INFINITY;               // every score left out of the candidates is <= l_drop
   float tau_c = 0.0f;                      // current evaluation point / final tau
   int iter = 0;
   bool row_done = false;                   // threshold certified exact
   float rowsum = 0.0f;
 
   auto trace_store = [&](int it, float val) {
-    if (P.tau_trace != nullptr && row_ok)
+    if (P.tau_trace != nullptr && row_ok && it <= P.max_iter)
       P.tau_trace[(static_cast<size_t>(it) * P.BH + bh) * P.N + row] = val;
   };
 
@@ -296,6 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       double F0 = 0.0, F1 = 0.0, F2 = 0.0;  // refinement sums at tau_c
       float Tmin = INFINITY;                // smallest positive s - tau_c
+      float Tneg = -INFINITY;               // largest non-positive s - tau_c
       if (kind == PASS_PV) rowsum = 0.0f;
       for (int t = 0; t < n; ++t) {
         const int j = sm.tiles[t];
@@ -310,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         if (kind == PASS_HIST) {
           float tile_max = -INFINITY;
+          float cmx0 = -INFINITY, cmx1 = -INFINITY, cmx2 = -INFINITY, cmx3 = -INFINITY;
 #pragma unroll 1
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t r[32];
@@ -318,10 +458,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (msk) apply_mask(v, j, ch);
-            float cm = v[0];
-#pragma unroll
-            for (int e = 1; e < 32; ++e) cm = fmaxf(cm, v[e]);
+            const float cm = max32(v);
             tile_max = fmaxf(tile_max, cm);
+            m_raw = fmaxf(m_raw, cm);
             if (cm > -INFINITY) {
               const int gc = static_cast<int>(
                   __float_as_uint(__fmaf_rd(fmaxf(cm, -P.slim), P.cN, kMagic)) - kMagicBits);
@@ -358,15 +497,91 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int b = 0; b <= kNB; ++b)
                 cnt[b] += static_cast<uint32_t>(packed >> (7 * b)) & 127u;
             }
+            if (ch == 0) cmx0 = cm;
+            else if (ch == 1) cmx1 = cm;
+            else if (ch == 2) cmx2 = cm;
+            else cmx3 = cm;
+          }
+          // Candidates of this tile: every score above acc_raw, a lower bound of
+          // tau* (the running max - 1, raised to the partial histogram's tau_h
+          // -- tau_h of the scores seen so far, this tile included -- whenever
+          // some chunk of the tile reaches the current bound).
+          {
+            const float cmt = fmaxf(fmaxf(cmx0, cmx1), fmaxf(cmx2, cmx3));
+            acc_raw = fmaxf(acc_raw, __fsub_rd(m_raw, P.inv_c));
+            if (row_ok && !cand_over && gtop_set && cmt > acc_raw) {
+              const double th = hist_threshold<ALPHA2>(cnt, gtop);
+              acc_raw = fmaxf(acc_raw, __double2float_rd((th - hist_margin(th)) / P.c));
+            }
+          }
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            const float cm = ch == 0 ? cmx0 : ch == 1 ? cmx1 : ch == 2 ? cmx2 : cmx3;
+            const bool want = row_ok && !cand_over && cm > acc_raw;
+            if (!__any_sync(0xffffffffu, want)) continue;
+            uint32_t r[32];
+            tmem_ld32(t_s + ch * 32, r);
+            if (!want) continue;
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+            if (msk) apply_mask(v, j, ch);
+            if (ncand + 32 > kCap) {
+              if (prunes < kMaxPrunes) {
+                // drop the listed scores that fell below the bound
+                ++prunes;
+                int kept = 0;
+                for (int a = 0; a < ncand; ++a) {
+                  const float xa = my_cand[a * kTile];
+                  if (xa > acc_raw) my_cand[(kept++) * kTile] = xa;
+                }
+                ncand = kept;
+              }
+              cand_over = ncand + 32 > kCap;
+            }
+            if (!cand_over) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                if (v[e] > acc_raw) my_cand[(ncand++) * kTile] = v[e];
+              }
+            }
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
-          m_raw = fmaxf(m_raw, tile_max);
           const float rec = row_ok ? tile_max * P.c : -INFINITY;
           P.tmax[tmax_index(bh, i, j, P.tr, P.tc, P.causal) + rl] = __float2half_ru(rec);
+        } else if (kind == PASS_COLLECT) {
+          // rebuild the lists of the rows that overflowed: exactly the scores above lo
+          const float thr = collect ? __double2float_rd(lo / P.c) : INFINITY;
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(t_s + ch * 32, r);
+            if (ch == 3) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+            }
+            if (!collect) continue;
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+            if (msk) apply_mask(v, j, ch);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (v[e] > thr) {
+                if (ncand < kCap) my_cand[ncand * kTile] = v[e];
+                ++ncand;
+              }
+            }
+          }
         } else if (kind == PASS_REFINE) {
-          float f0 = 0.f, f1 = 0.f, f2 = 0.f, tmin = INFINITY;
+          // four independent partial accumulators per quantity (ILP)
+          float f0[4] = {0.f, 0.f, 0.f, 0.f}, f1[4] = {0.f, 0.f, 0.f, 0.f},
+                f2[4] = {0.f, 0.f, 0.f, 0.f};
+          float tmin[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+          float tneg[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t r[32];
@@ -377,27 +592,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (msk) apply_mask(v, j, ch);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
+              const int a = e & 3;
               const float tt = fmaf(v[e], P.c, -tau_c);
               const bool in = tt > 0.0f;
               const float tp = fmaxf(tt, 0.0f);
-              tmin = in ? fminf(tmin, tt) : tmin;
+              tmin[a] = in ? fminf(tmin[a], tt) : tmin[a];
+              tneg[a] = in ? tneg[a] : fmaxf(tneg[a], tt);
               if (ALPHA2) {
-                f0 += tp;
-                f1 += in ? 1.0f : 0.0f;
+                f0[a] += tp;
+                f1[a] += in ? 1.0f : 0.0f;
               } else {
-                f0 = fmaf(tp, tp, f0);
-                f1 += tp;
-                f2 += in ? 1.0f : 0.0f;
+                f0[a] = fmaf(tp, tp, f0[a]);
+                f1[a] += tp;
+                f2[a] += in ? 1.0f : 0.0f;
               }
             }
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
-          F0 += f0;
-          F1 += f1;
-          F2 += f2;
-          Tmin = fminf(Tmin, tmin);
+          F0 += (f0[0] + f0[1]) + (f0[2] + f0[3]);
+          F1 += (f1[0] + f1[1]) + (f1[2] + f1[3]);
+          F2 += (f2[0] + f2[1]) + (f2[2] + f2[3]);
+          Tmin = fminf(Tmin, fminf(fminf(tmin[0], tmin[1]), fminf(tmin[2], tmin[3])));
+          Tneg = fmaxf(Tneg, fmaxf(fmaxf(tneg[0], tneg[1]), fmaxf(tneg[2], tneg[3])));
         } else {  // PASS_PV
           const uint32_t cur_p = pc++;
           if (cur_p > 0) {
@@ -421,17 +639,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (msk) apply_mask(v, j, ch);
             uint32_t w[16];
-            float psum = 0.f;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const float t0 = fmaxf(fmaf(v[2 * e], P.c, -tau_c), 0.0f);
               const float t1 = fmaxf(fmaf(v[2 * e + 1], P.c, -tau_c), 0.0f);
               const float p0 = ALPHA2 ? t0 : t0 * t0;
               const float p1 = ALPHA2 ? t1 : t1 * t1;
-              psum += p0 + p1;
+              ps[e & 3] += p0 + p1;
               const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
               w[e] = *reinterpret_cast<const uint32_t*>(&h2);
             }
+            const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
             if (ch < 2) part_lo += psum; else part_hi += psum;
 #pragma unroll
             for (int qd = 0; qd < 4; ++qd) {
@@ -480,129 +699,121 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
+      // Refinement over the row's candidate list (every score that can be in
+      // the support), in registers: no further pass over the keys.
+      auto refine_registers = [&]() {
+        // only once the list holds every score above lo: after HIST for rows
+        // whose list never overflowed, after COLLECT for the rebuilt ones
+        if (!row_ok || cand_over || (collect && kind == PASS_HIST)) return;
+        for (; iter < P.max_iter && !row_done;) {
+          float f0[4] = {0.f, 0.f, 0.f, 0.f}, f1[4] = {0.f, 0.f, 0.f, 0.f},
+                f2[4] = {0.f, 0.f, 0.f, 0.f};
+          float tmn[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+          float tng[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          for (int e0 = 0; e0 < ncand; e0 += 4) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              const float tt =
+                  e0 + a < ncand ? fmaf(my_cand[(e0 + a) * kTile], P.c, -tau_c) : -INFINITY;
+              const bool in = tt > 0.0f;
+              const float tp = fmaxf(tt, 0.0f);
+              tmn[a] = in ? fminf(tmn[a], tt) : tmn[a];
+              tng[a] = in ? tng[a] : fmaxf(tng[a], tt);
+              if (ALPHA2) {
+                f0[a] += tp;
+                f1[a] += in ? 1.0f : 0.0f;
+              } else {
+                f0[a] = fmaf(tp, tp, f0[a]);
+                f1[a] += tp;
+                f2[a] += in ? 1.0f : 0.0f;
+              }
+            }
+          }
+          const double F0c = (f0[0] + f0[1]) + (f0[2] + f0[3]);
+          const double F1c = (f1[0] + f1[1]) + (f1[2] + f1[3]);
+          const double F2c = (f2[0] + f2[1]) + (f2[2] + f2[3]);
+          const float tminc = fminf(fminf(tmn[0], tmn[1]), fminf(tmn[2], tmn[3]));
+          const float tnegc = fmaxf(fmaxf(tng[0], tng[1]), fmaxf(tng[2], tng[3]));
+          row_done = solver_step<ALPHA2>(F0c, F1c, F2c, tminc, tnegc, l_drop, tau_c, lo, hi);
+          ++iter;
+          trace_store(iter, tau_c);
+        }
+      };
+      // Publish the next pass: PV unless some row still needs its list rebuilt
+      // (COLLECT) or must refine over the key tiles (REFINE).
+      auto next_pass = [&](int passes_done_kind) {
+        // the candidate slots are V-ring / P-tile memory that TMA and the
+        // tensor core use next: order these generic accesses before them
+        fence_proxy_async_smem();
+        build_list(lo);
+        epi_bar();
+        if (warp == 2) {
+          const int nn = compact_tiles(sm.flags, (ntc + 31) >> 5, sm.tiles);
+          if (lane == 0) {
+            sm.ctl_n = nn;
+            int next = PASS_PV;
+            if (sm.cand_overflow == 1) next = PASS_COLLECT;
+            else if (sm.cand_overflow == 2 && sm.ctl_iter < P.max_iter && sm.not_converged)
+              next = PASS_REFINE;
+            sm.ctl_kind = next;
+            sm.not_converged = 0;
+            atomicAdd(&P.counters[passes_done_kind], static_cast<unsigned long long>(n));
+            if (passes_done_kind == CNT_REFINE_TILES) atomicAdd(&P.counters[CNT_REFINE_PASSES], 1ull);
+          }
+        }
+      };
+
       if (kind == PASS_HIST) {
         double tau_h = 0.0;
         if (row_ok) {
           if (fabsf(m_raw * P.cN) >= 2097152.0f) atomicOr(P.status, ST_RANGE);
-          // Reduced problem sum_b cnt_b [x_b - tau]_+^k = 1 with x_b = b / kNB
-          // (relative to the window base): scan candidate supports from the
-          // top bin down and take the first closed-form root that does not
-          // reach the next lower bin.
-          double C = 0.0, S1 = 0.0, S2 = 0.0, rel = 0.0;
-          bool found = false;
-#pragma unroll
-          for (int b = kNB; b >= 0; --b) {
-            const double cb = static_cast<double>(cnt[b]);
-            const double x = static_cast<double>(b) / kNB;
-            C += cb;
-            S1 += cb * x;
-            S2 += cb * x * x;
-            if (!found && C > 0.0) {
-              double cand;
-              bool valid = true;
-              if (ALPHA2) {
-                cand = (S1 - 1.0) / C;
-              } else {
-                const double disc = S1 * S1 - C * (S2 - 1.0);
-                valid = disc >= 0.0;
-                cand = (S1 - sqrt(fmax(disc, 0.0))) / C;
-              }
-              const double lower = (b == 0) ? -1e300 : static_cast<double>(b - 1) / kNB;
-              if (valid && cand >= lower) {
-                rel = cand;
-                found = true;
-              }
-            }
-          }
-          tau_h = static_cast<double>(gtop - kNB) / kNB + rel;
-          const double margin = 9.5367431640625e-07 * fmax(1.0, fabs(tau_h));  // 2^-20
+          tau_h = hist_threshold<ALPHA2>(cnt, gtop);
+          const double margin = hist_margin(tau_h);
           const double m_s = static_cast<double>(m_raw) * P.c;
           const double nb = ALPHA2 ? 1.0 / n_valid : 1.0 / sqrt(static_cast<double>(n_valid));
           lo = tau_h - margin;
           hi = fmin(tau_h + 1.0 / kNB + margin, m_s - nb + margin);
+          l_drop = static_cast<double>(acc_raw) * P.c;   // every unlisted score is <= l_drop <= tau*
+          lo = fmax(lo, l_drop);
           if (hi < lo) hi = lo;
           tau_c = __double2float_rd(lo);
           lo = tau_c;
+          if (cand_over && P.max_iter > 0) {
+            // the list lost scores: rebuild it above lo in a COLLECT pass
+            collect = true;
+            cand_over = false;
+            ncand = 0;
+            l_drop = lo;
+            sm.cand_overflow = 1;
+          }
         }
         iter = 0;
         trace_store(0, static_cast<float>(tau_h));
-        build_list(lo);
         epi_bar();
-        if (warp == 2) {
-          const int nn = compact_tiles(sm.flags, (ntc + 31) >> 5, sm.tiles);
-          if (lane == 0) {
-            sm.ctl_n = nn;
-            sm.ctl_kind = P.max_iter > 0 ? PASS_REFINE : PASS_PV;
-            atomicAdd(&P.counters[CNT_HIST_TILES], static_cast<unsigned long long>(n));
-          }
+        refine_registers();
+        next_pass(CNT_HIST_TILES);
+        if (warp == 2 && lane == 0 && sm.ctl_kind == PASS_COLLECT)
+          atomicAdd(&P.counters[CNT_CAND_OVERFLOW], 1ull);
+      } else if (kind == PASS_COLLECT) {
+        if (row_ok && collect) {
+          cand_over = ncand > kCap;
+          if (cand_over) sm.cand_overflow = 2;   // refine this tile over the key tiles
         }
+        epi_bar();
+        if (warp == 2 && lane == 0 && sm.cand_overflow == 1) sm.cand_overflow = 0;
+        epi_bar();
+        refine_registers();
+        if (row_ok && !row_done && iter < P.max_iter) sm.not_converged = 1;
+        next_pass(CNT_REFINE_TILES);
       } else if (kind == PASS_REFINE) {
-        if (row_ok && !row_done) {
-          // f(tau) = sum_i [s_i - tau]_+^k - 1 at tau_c: F0 = sum t^k,
-          // F1 = sum t^(k-1), F2 = sum t^(k-2) (alpha = 1.5: k = 2; alpha = 2: k = 1).
-          const double f = F0 - 1.0;
-          if (f > 0.0) lo = fmax(lo, static_cast<double>(tau_c));
-          else if (f < 0.0) hi = fmin(hi, static_cast<double>(tau_c));
-          double tn = 0.5 * (lo + hi);
-          bool exact = (f == 0.0);
-          if (exact) {
-            tn = tau_c;
-          } else if (ALPHA2) {
-            // Newton: f is convex and piecewise linear, so the tangent root is a
-            // lower bound of tau*; it is tau* itself when no score of the
-            // current support is crossed (step < smallest positive gap).
-            if (F1 > 0.0) {
-              const double d = f / F1;
-              tn = tau_c + d;
-              lo = fmax(lo, tn);
-              exact = f > 0.0 && d < static_cast<double>(Tmin);
-            }
-          } else {
-            if (F1 > 0.0) {
-              // Newton lower bound (f convex).
-              lo = fmax(lo, tau_c + f / (2.0 * F1));
-              // On the current support f is the quadratic F2 d^2 - 2 F1 d + F0 - 1
-              // in d = tau - tau_c.  Its smaller root is tau* if it does not
-              // cross a support score, and an upper bound of tau* otherwise.
-              const double disc = F1 * F1 - F2 * f;
-              if (f > 0.0 && disc >= 0.0 && F2 > 0.0) {
-                const double dq = (F1 - sqrt(disc)) / F2;
-                if (dq <= static_cast<double>(Tmin)) {
-                  tn = tau_c + dq;
-                  exact = true;
-                } else {
-                  hi = fmin(hi, tau_c + dq);
-                }
-              }
-              if (!exact) {
-                const double fp = -2.0 * F1, fpp = 2.0 * F2;
-                tn = tau_c - 2.0 * f * fp / (2.0 * fp * fp - f * fpp);  // Halley
-              }
-            }
-          }
-          if (!exact && !(tn >= lo && tn <= hi)) tn = 0.5 * (lo + hi);  // bisection fallback
-          tau_c = static_cast<float>(tn);
-          if (exact) {
-            row_done = true;
-            lo = fmax(lo, static_cast<double>(__double2float_rd(tn)));
-          } else {
-            sm.not_converged = 1;
-          }
+        if (row_ok && !row_done && iter < P.max_iter) {
+          row_done = solver_step<ALPHA2>(F0, F1, F2, Tmin, Tneg, l_drop, tau_c, lo, hi);
+          ++iter;
+          trace_store(iter, tau_c);
+          if (!row_done && iter < P.max_iter) sm.not_converged = 1;
         }
-        ++iter;
-        trace_store(iter, tau_c);
-        build_list(lo);
-        epi_bar();
-        if (warp == 2) {
-          const int nn = compact_tiles(sm.flags, (ntc + 31) >> 5, sm.tiles);
-          if (lane == 0) {
-            sm.ctl_n = nn;
-            sm.ctl_kind = (iter < P.max_iter && sm.not_converged) ? PASS_REFINE : PASS_PV;
-            sm.not_converged = 0;
-            atomicAdd(&P.counters[CNT_REFINE_TILES], static_cast<unsigned long long>(n));
-            atomicAdd(&P.counters[CNT_REFINE_PASSES], 1ull);
-          }
-        }
+        if (warp == 2 && lane == 0) ++sm.ctl_iter;
+        next_pass(CNT_REFINE_TILES);
       } else {  // PASS_PV: write O, tau, mask
         if (ok && n > 0) {
           ok = mbar_wait(&sm.o_full, 0, abort_flag, P.status);

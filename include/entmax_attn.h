@@ -86,8 +86,9 @@ int entmax_attn_mask_words(int N, int block);
  * Bytes of device workspace that entmax_attn_fwd and entmax_attn_bwd need for
  * this problem (the same buffer serves both).  It holds the status word and
  * work counters, the per-(row, key tile) score maxima of the histogram pass
- * (fp16, rounded up), the tile-granularity mask and its transpose, the per-row
- * delta of the backward and the backward's fp16 copies of q, k, v and dout.
+ * (fp16, rounded up), the tile-granularity mask and its transpose, the
+ * per-row delta of the backward and the backward's fp16 copies of q, k, v and
+ * dout.
  * Returns 0 for unsupported arguments.
  */
 size_t entmax_attn_workspace_size(int B, int H, int N, int D, int block, int causal);
@@ -186,11 +187,13 @@ int entmax_attn_status(const void* workspace, void* stream, uint32_t* status);
 /*
  * Diagnostics: copies the first n (1..8) work counters of `workspace` to
  * counters[] after synchronising `stream`.  [0] key tiles visited by the
- * forward's histogram pass, [1] by its refinement passes, [2] by its P.V pass,
- * [3] refinement passes summed over 128-row tiles, [4] active key tiles per
- * pass of the backward row kernel, [5] active query tiles of the backward
- * column kernel (tiles are 128 x 128).  Cleared by entmax_attn_fwd ([0]-[3])
- * and entmax_attn_bwd ([4]-[5]).
+ * forward's histogram pass, [1] by its tile refinement passes, [2] by its P.V
+ * pass, [3] tile refinement passes summed over 128-row tiles, [4] active key
+ * tiles per pass of the backward row kernel, [5] active query tiles of the
+ * backward column kernel, [6] 128-row tiles whose candidate lists overflowed
+ * (and which therefore refined by streaming the key tiles again); tiles are
+ * 128 x 128.  Cleared by entmax_attn_fwd ([0]-[3], [6]) and entmax_attn_bwd
+ * ([4]-[5]).
  */
 int entmax_attn_counters(const void* workspace, void* stream, unsigned long long* counters, int n);
 

@@ -64,6 +64,26 @@ def test_histogram_bound_and_iterations(cuda_device, alpha):
         assert frac[2] >= 0.95
 
 
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_all_equal_scores_overflow_path(cuda_device, alpha):
+    """q = 0 makes every visible score equal: each row is uniform over its
+    n visible keys with tau = -n^(1-alpha).  Every score is a candidate, so the
+    per-row candidate lists overflow and the tile refinement passes run."""
+    import differentiable_sparse_attention_b200 as dsa
+    w = Workload("equal", B=1, H=2, N=384, D=64, alpha=alpha, seed=4)
+    x = make_inputs(w, device=cuda_device, need_grad_inputs=False)
+    q = torch.zeros_like(x["q"])
+    res = entmax_attn_fwd(q, x["k"], x["v"], alpha, True, 128)
+    assert status(res.workspace) == 0
+    assert dsa.counters(res.workspace)["fwd_cand_overflow_tiles"] > 0
+    for h in range(2):
+        check_forward_head(res, 0, h, to64(q, 0, h), to64(x["k"], 0, h), to64(x["v"], 0, h),
+                           alpha, True, 128)
+    n = np.arange(1, 385, dtype=np.float64)
+    np.testing.assert_allclose(res.tau[0, 0].cpu().numpy(), -n ** (1 - alpha), rtol=0,
+                               atol=1e-5)
+
+
 def test_max_iter_zero_raises_status(cuda_device):
     w = Workload("noiter", B=1, H=1, N=256, D=64, alpha=1.5, temperature=1.0, seed=1)
     x = make_inputs(w, device=cuda_device, need_grad_inputs=False)

@@ -14,6 +14,7 @@
 #include "entmax_attn.h"
 #include "fwd.cuh"
 #include "bwd.cuh"
+#include "simt32.cuh"
 
 using namespace entmax;
 
@@ -60,7 +61,8 @@ int check_common(int B, int H, int N, int D, int dtype, float alpha, int block) 
   if (B < 1 || H < 1 || N < 1 || N > kMaxN) return ENTMAX_E_SHAPE;
   if (static_cast<long long>(B) * H * ((N + kTile - 1) / kTile) > 0x7fffffffLL) return ENTMAX_E_SHAPE;
   if (D != 64 && D != 128) return ENTMAX_E_UNSUPPORTED;
-  if (dtype != ENTMAX_DTYPE_BF16) return ENTMAX_E_UNSUPPORTED;
+  if (dtype != ENTMAX_DTYPE_BF16 && dtype != ENTMAX_DTYPE_FP32) return ENTMAX_E_UNSUPPORTED;
+  if (dtype == ENTMAX_DTYPE_FP32 && D != kF32D) return ENTMAX_E_UNSUPPORTED;
   if (block != 64 && block != 128) return ENTMAX_E_UNSUPPORTED;
   if (!(alpha == 1.5f || alpha == 2.0f)) return ENTMAX_E_ALPHA;
   return ENTMAX_OK;
@@ -184,6 +186,47 @@ void* noalloc_scratch_ptr(int device) {
   return ptrs[device];
 }
 
+F32Params make_f32_params(int B, int H, int N, int D, float alpha, int causal, int block,
+                          int max_iter, uint8_t* ws, const WsLayout& L) {
+  F32Params p{};
+  p.BH = B * H;
+  p.N = N;
+  p.causal = causal ? 1 : 0;
+  p.block = block;
+  p.mask_rows = (N + block - 1) / block;
+  p.mask_words = (p.mask_rows + 31) / 32;
+  p.max_iter = max_iter;
+  p.c = (alpha - 1.0f) / std::sqrt(static_cast<float>(D));
+  p.cN = p.c * static_cast<float>(kNB);
+  p.slim = 2097152.0f / p.cN;
+  p.inv_c = std::nextafter(1.0f / p.c, INFINITY) * (1.0f + 1e-6f);
+  p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(D));
+  p.delta = reinterpret_cast<float*>(ws + L.delta);
+  p.status = reinterpret_cast<uint32_t*>(ws + L.status);
+  p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
+  return p;
+}
+
+template <bool A2>
+int launch_fwd_f32(const F32Params& p, cudaStream_t st) {
+  auto kern = entmax_fwd_f32_kernel<A2>;
+  static bool attr_ok = set_smem(kern, kF32CandBytes);
+  if (!attr_ok) return ENTMAX_E_CUDA;
+  dim3 grid((p.N + 127) / 128, p.BH);
+  kern<<<grid, 128, kF32CandBytes, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
+}
+
+template <bool A2>
+int launch_bwd_f32(const F32Params& p, cudaStream_t st) {
+  dim3 grid((p.N + 63) / 64, p.BH);
+  entmax_bwd_row_f32_kernel<A2><<<grid, 128, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ENTMAX_E_CUDA;
+  prof_mark(EV_BWD_ROW, st);
+  entmax_bwd_col_f32_kernel<A2><<<grid, 128, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
+}
+
 }  // namespace
 
 // ============================================================== C ABI
@@ -218,13 +261,26 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
-    return ENTMAX_E_CUDA;
-
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   // status word + work counters live in the first 256 bytes
   if (cudaMemsetAsync(ws + L.status, 0, 8 + CNT_COUNT * sizeof(unsigned long long), st) != cudaSuccess)
+    return ENTMAX_E_CUDA;
+  if (dtype == ENTMAX_DTYPE_FP32) {
+    F32Params p = make_f32_params(B, H, N, D, alpha, causal, block, max_iter, ws, L);
+    p.q = static_cast<const float*>(q);
+    p.k = static_cast<const float*>(k);
+    p.v = static_cast<const float*>(v);
+    p.out = static_cast<float*>(out);
+    p.tau = tau;
+    p.mask = mask;
+    p.tau_trace = tau_trace;
+    prof_mark(EV_FWD0, st);
+    rc = alpha == 2.0f ? launch_fwd_f32<true>(p, st) : launch_fwd_f32<false>(p, st);
+    prof_mark(EV_FWD1, st);
+    return rc;
+  }
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
     return ENTMAX_E_CUDA;
 
   FwdParams p{};
@@ -341,6 +397,23 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
   if (cudaMemsetAsync(counters + CNT_ROW_TILES, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
     return ENTMAX_E_CUDA;
   prof_mark(EV_BWD0, st);
+  if (dtype == ENTMAX_DTYPE_FP32) {
+    F32Params p = make_f32_params(B, H, N, D, alpha, causal, block, 0, ws, L);
+    p.q = static_cast<const float*>(q);
+    p.k = static_cast<const float*>(k);
+    p.v = static_cast<const float*>(v);
+    p.dout = static_cast<const float*>(dout);
+    p.tau = const_cast<float*>(tau);
+    p.mask = const_cast<uint32_t*>(mask);
+    p.dq = static_cast<float*>(dq);
+    p.dk = static_cast<float*>(dk);
+    p.dv = static_cast<float*>(dv);
+    prof_mark(EV_BWD_CONV, st);
+    prof_mark(EV_BWD_MASK, st);
+    rc = alpha == 2.0f ? launch_bwd_f32<true>(p, st) : launch_bwd_f32<false>(p, st);
+    prof_mark(EV_BWD_COL, st);
+    return rc;
+  }
   const size_t elems = static_cast<size_t>(BH) * N * D;
   __half* h16[4];
   const void* srcs[4] = {q, k, v, dout};

@@ -38,7 +38,8 @@
  *     OR-ed into a status word at the start of the workspace; read it with
  *     entmax_attn_status().  Kernels never trap.
  *   - Supported: D in {64, 128}; block in {64, 128}; alpha in {1.5, 2.0};
- *     1 <= N <= ENTMAX_MAX_N; dtype bf16 (tensor-core path) or fp32.
+ *     1 <= N <= ENTMAX_MAX_N; dtype bf16 (tcgen05 tensor-core path) or fp32
+ *     (CUDA-core path for full fp32 precision, D = 64 only).
  */
 #ifndef ENTMAX_ATTN_H
 #define ENTMAX_ATTN_H

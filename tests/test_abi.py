@@ -64,6 +64,7 @@ def test_forward_argument_validation(lib):
     assert fwd(lib, D=96) == dsa.E_UNSUPPORTED
     assert fwd(lib, block=32) == dsa.E_UNSUPPORTED
     assert fwd(lib, dtype=7) == dsa.E_UNSUPPORTED
+    assert fwd(lib, dtype=1, D=128) == dsa.E_UNSUPPORTED   # fp32 path: head dim 64
     assert fwd(lib, alpha=1.0) == dsa.E_ALPHA
     assert fwd(lib, alpha=1.7) == dsa.E_ALPHA
     assert fwd(lib, max_iter=-1) == dsa.E_MAXITER

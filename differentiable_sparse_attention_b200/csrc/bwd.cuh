@@ -140,6 +140,18 @@ __device__ __forceinline__ int load_tile_list(const uint32_t* rowbits, int wt, u
   return total;
 }
 
+// Both backward kernels work in half-tile steps: a 128 x 128 tile is two
+// 64-column steps, so the S / dP accumulators fit twice in TMEM (double
+// buffering) and the MMAs of one half overlap the epilogue of the other.
+// Two epilogue warpgroups (warps 2-5 and 6-9) alternate: warpgroup h owns half
+// h of every tile and its TMEM / SMEM buffer.
+constexpr int kBwdThreads = 320;
+constexpr int kBwdEpi = 256;
+constexpr int kHalf = 64;
+constexpr int kHalfBytes = kTile * kHalf * 2;   // one [128][64] fp16 slab
+
+__device__ __forceinline__ void bwd_epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 // ============================================================ row kernel (delta, dQ)
 template <int D, int NSK, int NSV>
 struct BwdRowSmem {
@@ -147,11 +159,13 @@ struct BwdRowSmem {
   __half dout[kTile * D];
   __half k[NSK][kTile * D];
   __half v[NSV][kTile * D];
-  __half ds[kTile * kTile];   // dS tile, K-major (K = keys)
+  __half ds[2][kTile * kHalf];       // dS half tiles [128 rows][64 keys], K-major
+  float part_gdp[2][kTile];          // pass-A partial sums per warpgroup
+  float part_g[2][kTile];
   uint64_t qdo_full;
   uint64_t k_full[NSK], k_empty[NSK];
   uint64_t v_full[NSV], v_empty[NSV];
-  uint64_t s_full, s_empty, ds_full, ds_empty, dq_full, drain;
+  uint64_t s_full[2], s_empty[2], ds_full[2], ds_empty[2], dq_full, drain;
   uint32_t tmem_base;
   int abort_flag;
   int ntiles;
@@ -164,7 +178,7 @@ constexpr size_t bwd_row_smem_bytes() {
 }
 
 template <int D, int NSK, int NSV, bool ALPHA2>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     entmax_bwd_row_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
@@ -174,9 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto& sm = *reinterpret_cast<BwdRowSmem<D, NSK, NSV>*>(align1024(smem_raw));
   constexpr int kSlabs = D / 64;
   constexpr uint32_t kTileBytes = kTile * D * 2;
-  constexpr uint32_t kIdescS = make_idesc(kTile, kTile, 0, 0, 0, 0);  // [128 x D] x [128 x D]^T, f16
-  constexpr uint32_t kIdescDQ = make_idesc(kTile, D, 0, 0, 0, 1);     // dS (K-major) x K (MN-major)
-  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+  constexpr uint32_t kIdescS = make_idesc(kTile, kHalf, 0, 0, 0, 0);  // [128 x D] x [64 x D]^T
+  constexpr uint32_t kIdescDQ = make_idesc(kTile, D, 0, 0, 0, 1);     // dS half x K half (MN-major)
+  constexpr uint32_t kColDQ = 256;  // TMEM: buffer b holds S at 128 b, dP at 128 b + 64
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -187,10 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.qdo_full, 1);
     for (int s = 0; s < NSK; ++s) { mbar_init(&sm.k_full[s], 1); mbar_init(&sm.k_empty[s], 1); }
     for (int s = 0; s < NSV; ++s) { mbar_init(&sm.v_full[s], 1); mbar_init(&sm.v_empty[s], 1); }
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.s_empty, 4);
-    mbar_init(&sm.ds_full, 4);
-    mbar_init(&sm.ds_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_empty[b], 4);
+      mbar_init(&sm.ds_full[b], 4);
+      mbar_init(&sm.ds_empty[b], 1);
+    }
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -216,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t kc = 0, vc = 0;
 
   if (warp == 0) {
+    // ---------------------------------------------------------------- producer
     if (lane == 0) {
       bool ok = true;
       mbar_expect_tx(&sm.qdo_full, 2 * kTileBytes);
@@ -247,121 +264,129 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(&sm.qdo_full, 0, abort_flag, P.status);
       const uint32_t q_addr = smem_u32(sm.q), do_addr = smem_u32(sm.dout);
-      uint32_t sc = 0, dc = 0;
-      uint32_t kslot_prev = 0;
-      // S = Q K^T and dP = dO V^T of the next tile into TMEM.
+      uint32_t step = 0, dstep = 0;     // half-tile steps issued (S/dP) and dQ steps issued
+      uint32_t kcm = 0, vcm = 0;        // K / V tiles consumed
+      uint32_t ks_of0 = 0, ks_of1 = 0;  // K slot of the tile each buffer's step belongs to
+      // S = Q K_h^T and dP = dO V_h^T of step `step` (half h of the current tile)
       auto issue_sdp = [&](bool release_k) -> bool {
-        const uint32_t ks = kc % NSK, vs = vc % NSV;
-        if (!mbar_wait(&sm.k_full[ks], (kc / NSK) & 1, abort_flag, P.status)) return false;
-        if (!mbar_wait(&sm.v_full[vs], (vc / NSV) & 1, abort_flag, P.status)) return false;
-        if (sc > 0 && !mbar_wait(&sm.s_empty, (sc - 1) & 1, abort_flag, P.status)) return false;
+        const uint32_t h = step & 1, use = step >> 1;
+        const uint32_t ks = kcm % NSK, vs = vcm % NSV;
+        if (h == 0) {
+          if (!mbar_wait(&sm.k_full[ks], (kcm / NSK) & 1, abort_flag, P.status)) return false;
+          if (!mbar_wait(&sm.v_full[vs], (vcm / NSV) & 1, abort_flag, P.status)) return false;
+        }
+        if (use > 0 && !mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm.k[ks]), v_addr = smem_u32(sm.v[vs]);
+        const uint32_t k_addr = smem_u32(sm.k[ks]) + h * (kHalf * 128);
+        const uint32_t v_addr = smem_u32(sm.v[vs]) + h * (kHalf * 128);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-          mma_f16_ss(tmem + kColS, smem_desc_sw128(q_addr + off, 16, 1024),
+          mma_f16_ss(tmem + 128 * h, smem_desc_sw128(q_addr + off, 16, 1024),
                      smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-          mma_f16_ss(tmem + kColDP, smem_desc_sw128(do_addr + off, 16, 1024),
+          mma_f16_ss(tmem + 128 * h + kHalf, smem_desc_sw128(do_addr + off, 16, 1024),
                      smem_desc_sw128(v_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sm.s_full);
-        mma_commit(&sm.v_empty[vs]);
-        if (release_k) mma_commit(&sm.k_empty[ks]);
-        kslot_prev = ks;
-        ++kc;
-        ++vc;
-        ++sc;
+        mma_commit(&sm.s_full[h]);
+        if (h == 0) ks_of0 = ks;
+        else ks_of1 = ks;
+        if (h == 1) {
+          mma_commit(&sm.v_empty[vs]);
+          if (release_k) mma_commit(&sm.k_empty[ks]);
+          ++kcm;
+          ++vcm;
+        }
+        ++step;
         return true;
       };
-      // dQ += dS K of the previous tile (K slot kslot).
-      auto issue_dq = [&](uint32_t kslot) -> bool {
-        if (!mbar_wait(&sm.ds_full, dc & 1, abort_flag, P.status)) return false;
+      // dQ += dS_h K_h for dQ step `dstep`
+      auto issue_dq = [&]() -> bool {
+        const uint32_t h = dstep & 1, use = dstep >> 1;
+        if (!mbar_wait(&sm.ds_full[h], use & 1, abort_flag, P.status)) return false;
         tc_fence_after();
-        const uint32_t ds_addr = smem_u32(sm.ds), k_addr = smem_u32(sm.k[kslot]);
+        const uint32_t ks = h == 0 ? ks_of0 : ks_of1;
+        const uint32_t ds_addr = smem_u32(sm.ds[h]);
+        const uint32_t k_addr = smem_u32(sm.k[ks]) + h * (kHalf * 128);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint32_t a_off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-          mma_f16_ss(tmem + kColDQ, smem_desc_sw128(ds_addr + a_off, 16, 1024),
+        for (int kk = 0; kk < kHalf / 16; ++kk) {
+          mma_f16_ss(tmem + kColDQ, smem_desc_sw128(ds_addr + kk * 32, 16, 1024),
                      smem_desc_sw128(k_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescDQ,
-                     (dc > 0 || kk > 0) ? 1u : 0u);
+                     (dstep > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&sm.ds_empty);
-        mma_commit(&sm.k_empty[kslot]);
-        ++dc;
+        mma_commit(&sm.ds_empty[h]);
+        if (h == 1) mma_commit(&sm.k_empty[ks]);
+        ++dstep;
         return true;
       };
       // pass A: delta
-      for (int t = 0; t < n && ok; ++t) ok = issue_sdp(true);
-      // pass B: dQ, software-pipelined by one tile
-      uint32_t pending = 0;
-      for (int t = 0; t <= n && ok; ++t) {
-        uint32_t this_slot = 0;
-        if (t < n) {
-          ok = issue_sdp(false);
-          this_slot = kslot_prev;
-        }
-        if (ok && t > 0) ok = issue_dq(pending);
-        pending = this_slot;
+      for (int u = 0; u < 2 * n && ok; ++u) ok = issue_sdp(true);
+      // pass B: dQ, dQ steps trail the S/dP steps by one
+      for (int u = 0; u <= 2 * n && ok; ++u) {
+        if (u < 2 * n) ok = issue_sdp(false);
+        if (ok && u > 0) ok = issue_dq();
       }
       if (ok) mma_commit(&sm.dq_full);
+      kc = kcm;
+      vc = vcm;
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
+    const int wg = (warp - 2) >> 2;        // warpgroup: owns half wg of every tile
     const int quad = warp & 3;
     const int rl = quad * 32 + lane;
     const int row = i * kTile + rl;
     const bool row_ok = row < P.N;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t t_s = t_lane + 128 * wg, t_dp = t_s + kHalf;
     const float tau_r = row_ok ? P.tau[static_cast<size_t>(bh) * P.N + row] : INFINITY;
     bool ok = true;
-    uint32_t sc = 0, dc = 0;
-    double gdp = 0.0, gsum = 0.0;
+    uint32_t use = 0;   // uses of this warpgroup's S/dP buffer
     float delta = 0.0f;
-    uint8_t* ds_base = reinterpret_cast<uint8_t*>(sm.ds);
-
-    auto valid_col = [&](int col) { return col < P.N && (!P.causal || col <= row); };
+    uint8_t* ds_base = reinterpret_cast<uint8_t*>(sm.ds[wg]);
 
     for (int pass = 0; pass < 2 && ok; ++pass) {
+      float gdp[4] = {0.f, 0.f, 0.f, 0.f}, gsm[4] = {0.f, 0.f, 0.f, 0.f};
       for (int t = 0; t < n; ++t) {
         const int j = sm.tiles[t];
-        ok = mbar_wait(&sm.s_full, sc & 1, abort_flag, P.status);
+        ok = mbar_wait(&sm.s_full[wg], use & 1, abort_flag, P.status);
+        // pass B, tile t >= 1: the dQ MMA of tile t - 1 must have read this dS buffer
+        if (ok && pass == 1 && use > static_cast<uint32_t>(n))
+          ok = mbar_wait(&sm.ds_empty[wg], (use - n - 1) & 1, abort_flag, P.status);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        ++sc;
+        ++use;
         tc_fence_after();
-        if (pass == 1 && dc > 0) {
-          ok = mbar_wait(&sm.ds_empty, (dc - 1) & 1, abort_flag, P.status);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-        }
-        const bool msk = (P.causal && j == i) || ((j + 1) * kTile > P.N);
-        float a_gdp[4] = {0.f, 0.f, 0.f, 0.f}, a_g[4] = {0.f, 0.f, 0.f, 0.f};
+        const int col0 = j * kTile + wg * kHalf;
+        const bool msk = (P.causal && j == i) || (col0 + kHalf > P.N);
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t rs[32], rp[32];
-          tmem_ld32x2(t_lane + kColS + ch * 32, rs, t_lane + kColDP + ch * 32, rp);
-          if (ch == 3) {
+          tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
+          if (ch == 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_empty);
+            if (lane == 0) mbar_arrive(&sm.s_empty[wg]);
           }
           float gg[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             float tt = fmaf(__uint_as_float(rs[e]), P.c, -tau_r);
-            if (msk && !valid_col(j * kTile + ch * 32 + e)) tt = -1.0f;
+            if (msk) {
+              const int col = col0 + ch * 32 + e;
+              if (!(col < P.N && (!P.causal || col <= row))) tt = -1.0f;
+            }
             gg[e] = ALPHA2 ? (tt > 0.f ? 1.f : 0.f) : fmaxf(tt, 0.f);
           }
           if (pass == 0) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              a_gdp[e & 3] = fmaf(gg[e], __uint_as_float(rp[e]), a_gdp[e & 3]);
-              a_g[e & 3] += gg[e];
+              gdp[e & 3] = fmaf(gg[e], __uint_as_float(rp[e]), gdp[e & 3]);
+              gsm[e & 3] += gg[e];
             }
           } else {
             uint32_t w[16];
@@ -378,22 +403,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                   make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
           }
         }
-        if (pass == 0) {
-          gdp += (a_gdp[0] + a_gdp[1]) + (a_gdp[2] + a_gdp[3]);
-          gsum += (a_g[0] + a_g[1]) + (a_g[2] + a_g[3]);
-        } else {
+        if (pass == 1) {
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.ds_full);
-          ++dc;
+          if (lane == 0) mbar_arrive(&sm.ds_full[wg]);
         }
       }
       if (pass == 0) {
-        delta = gsum > 0.0 ? static_cast<float>(gdp / gsum) : 0.0f;
-        if (row_ok) P.delta[static_cast<size_t>(bh) * P.N + row] = delta;
+        // combine the two warpgroups' partial sums of the row: delta = sum g dP / sum g
+        sm.part_gdp[wg][rl] = (gdp[0] + gdp[1]) + (gdp[2] + gdp[3]);
+        sm.part_g[wg][rl] = (gsm[0] + gsm[1]) + (gsm[2] + gsm[3]);
+        bwd_epi_bar();
+        const float a = sm.part_gdp[0][rl] + sm.part_gdp[1][rl];
+        const float g = sm.part_g[0][rl] + sm.part_g[1][rl];
+        delta = g > 0.f ? a / g : 0.0f;
+        if (row_ok && wg == 0) P.delta[static_cast<size_t>(bh) * P.N + row] = delta;
       }
     }
-    // dQ epilogue
+    // dQ epilogue: warpgroup wg stores columns [wg * D/2, (wg + 1) * D/2)
     if (ok && n > 0) {
       ok = mbar_wait(&sm.dq_full, 0, abort_flag, P.status);
       ok = __all_sync(0xffffffffu, ok);
@@ -401,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     __nv_bfloat16* dst_row = P.dq + (static_cast<size_t>(bh) * P.N + row) * D;
 #pragma unroll 1
-    for (int ch = 0; ch < D / 32; ++ch) {
+    for (int ch = wg * (D / 64); ch < (wg + 1) * (D / 64); ++ch) {
       uint32_t r[32];
       if (ok && n > 0) {
         tmem_ld32(t_lane + kColDQ + ch * 32, r);
@@ -454,13 +481,13 @@ struct BwdColSmem {
   __half v[kTile * D];
   __half q[NS][kTile * D];
   __half dout[NS][kTile * D];
-  __half pt[kTile * kTile];    // P^T tile  [keys][rows], K-major (K = rows)
-  __half dst[kTile * kTile];   // dS^T tile [keys][rows]
+  __half pt[2][kTile * kHalf];    // P^T half tiles  [128 keys][64 rows], K-major (K = rows)
+  __half dst[2][kTile * kHalf];   // dS^T half tiles [128 keys][64 rows]
   float tau[NS][kTile];
   float delta[NS][kTile];
   uint64_t kv_full;
   uint64_t q_full[NS], q_empty[NS];
-  uint64_t s_full, s_empty, pt_full, pt_empty, acc_full, drain;
+  uint64_t s_full[2], s_empty[2], pt_full[2], pt_empty[2], acc_full, drain;
   uint32_t tmem_base;
   int abort_flag;
   int ntiles;
@@ -473,7 +500,7 @@ constexpr size_t bwd_col_smem_bytes() {
 }
 
 template <int D, int NS, bool ALPHA2>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     entmax_bwd_col_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
@@ -482,9 +509,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto& sm = *reinterpret_cast<BwdColSmem<D, NS>*>(align1024(smem_raw));
   constexpr int kSlabs = D / 64;
   constexpr uint32_t kTileBytes = kTile * D * 2;
-  constexpr uint32_t kIdescS = make_idesc(kTile, kTile, 0, 0, 0, 0);   // K Q^T, V dO^T, f16
-  constexpr uint32_t kIdescAcc = make_idesc(kTile, D, 0, 0, 0, 1);    // P^T dO, dS^T Q
-  constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  constexpr uint32_t kIdescS = make_idesc(kTile, kHalf, 0, 0, 0, 0);   // K Q_h^T, V dO_h^T
+  constexpr uint32_t kIdescAcc = make_idesc(kTile, D, 0, 0, 0, 1);    // P^T_h dO_h, dS^T_h Q_h
+  constexpr uint32_t kColDV = 256, kColDK = 256 + D;  // buffer b: S^T at 128 b, dP^T at 128 b + 64
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -498,10 +525,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.q_full[s], 1 + 32);  // TMA expect_tx + 32 lanes staging tau/delta
       mbar_init(&sm.q_empty[s], 1);
     }
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.s_empty, 4);
-    mbar_init(&sm.pt_full, 4);
-    mbar_init(&sm.pt_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_empty[b], 4);
+      mbar_init(&sm.pt_full[b], 4);
+      mbar_init(&sm.pt_empty[b], 1);
+    }
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -570,94 +599,94 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       bool ok = mbar_wait(&sm.kv_full, 0, abort_flag, P.status);
       const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
-      uint32_t sc = 0, ac = 0;
-      auto issue_s = [&](uint32_t slot, uint32_t use) -> bool {
-        if (!mbar_wait(&sm.q_full[slot], use & 1, abort_flag, P.status)) return false;
-        if (sc > 0 && !mbar_wait(&sm.s_empty, (sc - 1) & 1, abort_flag, P.status)) return false;
+      // step u = 2 t + h: half h (query rows 64 h .. 64 h + 63) of active query tile t
+      auto issue_s = [&](uint32_t u) -> bool {
+        const uint32_t t = u >> 1, h = u & 1, slot = t % NS, use = u >> 1;
+        if (h == 0 && !mbar_wait(&sm.q_full[slot], (t / NS) & 1, abort_flag, P.status)) return false;
+        if (use > 0 && !mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sm.q[slot]), do_addr = smem_u32(sm.dout[slot]);
+        const uint32_t q_addr = smem_u32(sm.q[slot]) + h * (kHalf * 128);
+        const uint32_t do_addr = smem_u32(sm.dout[slot]) + h * (kHalf * 128);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-          mma_f16_ss(tmem + kColS, smem_desc_sw128(k_addr + off, 16, 1024),
+          mma_f16_ss(tmem + 128 * h, smem_desc_sw128(k_addr + off, 16, 1024),
                      smem_desc_sw128(q_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-          mma_f16_ss(tmem + kColDP, smem_desc_sw128(v_addr + off, 16, 1024),
+          mma_f16_ss(tmem + 128 * h + kHalf, smem_desc_sw128(v_addr + off, 16, 1024),
                      smem_desc_sw128(do_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sm.s_full);
-        ++sc;
+        mma_commit(&sm.s_full[h]);
         return true;
       };
-      auto issue_acc = [&](uint32_t slot) -> bool {
-        if (!mbar_wait(&sm.pt_full, ac & 1, abort_flag, P.status)) return false;
+      auto issue_acc = [&](uint32_t u) -> bool {
+        const uint32_t t = u >> 1, h = u & 1, slot = t % NS, use = u >> 1;
+        if (!mbar_wait(&sm.pt_full[h], use & 1, abort_flag, P.status)) return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sm.q[slot]), do_addr = smem_u32(sm.dout[slot]);
-        const uint32_t pt_addr = smem_u32(sm.pt), ds_addr = smem_u32(sm.dst);
+        const uint32_t q_addr = smem_u32(sm.q[slot]) + h * (kHalf * 128);
+        const uint32_t do_addr = smem_u32(sm.dout[slot]) + h * (kHalf * 128);
+        const uint32_t pt_addr = smem_u32(sm.pt[h]), ds_addr = smem_u32(sm.dst[h]);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint32_t a_off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-          const uint32_t b_off = kk * 16 * 128;
-          const uint32_t acc = (ac > 0 || kk > 0) ? 1u : 0u;
-          mma_f16_ss(tmem + kColDV, smem_desc_sw128(pt_addr + a_off, 16, 1024),
-                     smem_desc_sw128(do_addr + b_off, kSlabBytes, 1024), kIdescAcc, acc);
-          mma_f16_ss(tmem + kColDK, smem_desc_sw128(ds_addr + a_off, 16, 1024),
-                     smem_desc_sw128(q_addr + b_off, kSlabBytes, 1024), kIdescAcc, acc);
+        for (int kk = 0; kk < kHalf / 16; ++kk) {
+          const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
+          mma_f16_ss(tmem + kColDV, smem_desc_sw128(pt_addr + kk * 32, 16, 1024),
+                     smem_desc_sw128(do_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescAcc, acc);
+          mma_f16_ss(tmem + kColDK, smem_desc_sw128(ds_addr + kk * 32, 16, 1024),
+                     smem_desc_sw128(q_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescAcc, acc);
         }
-        mma_commit(&sm.pt_empty);
-        mma_commit(&sm.q_empty[slot]);
-        ++ac;
+        mma_commit(&sm.pt_empty[h]);
+        if (h == 1) mma_commit(&sm.q_empty[slot]);
         return true;
       };
-      if (NS >= 2) {
-        for (int t = 0; t <= n && ok; ++t) {
-          if (t < n) ok = issue_s(t % NS, t / NS);
-          if (ok && t > 0) ok = issue_acc((t - 1) % NS);
-        }
-      } else {
-        for (int t = 0; t < n && ok; ++t) {
-          ok = issue_s(0, t);
-          if (ok) ok = issue_acc(0);
-        }
+      const uint32_t steps = 2u * static_cast<uint32_t>(n);
+      for (uint32_t u = 0; u <= steps && ok; ++u) {
+        // With one Q / dO stage the previous tile's last accumulation must free
+        // it before the next tile's first S^T step can be loaded.
+        const bool acc_first = NS == 1 && (u & 1) == 0;
+        if (acc_first && u > 0) ok = issue_acc(u - 1);
+        if (ok && u < steps) ok = issue_s(u);
+        if (ok && !acc_first && u > 0) ok = issue_acc(u - 1);
       }
       if (ok) mma_commit(&sm.acc_full);
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
+    const int wg = (warp - 2) >> 2;           // warpgroup: owns half wg of every tile
     const int quad = warp & 3;
     const int kl = quad * 32 + lane;          // key within the tile
     const int key = j * kTile + kl;
     const bool key_ok = key < P.N;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t t_s = t_lane + 128 * wg, t_dp = t_s + kHalf;
     bool ok = true;
-    uint32_t sc = 0, ac = 0;
-    uint8_t* pt_base = reinterpret_cast<uint8_t*>(sm.pt);
-    uint8_t* ds_base = reinterpret_cast<uint8_t*>(sm.dst);
+    uint8_t* pt_base = reinterpret_cast<uint8_t*>(sm.pt[wg]);
+    uint8_t* ds_base = reinterpret_cast<uint8_t*>(sm.dst[wg]);
     for (int t = 0; t < n; ++t) {
       const int it = sm.tiles[t];
-      const uint32_t slot = t % NS, use = t / NS;
-      ok = mbar_wait(&sm.s_full, sc & 1, abort_flag, P.status) &&
-           mbar_wait(&sm.q_full[slot], use & 1, abort_flag, P.status);
-      if (ok && ac > 0) ok = mbar_wait(&sm.pt_empty, (ac - 1) & 1, abort_flag, P.status);
+      const uint32_t slot = t % NS;
+      ok = mbar_wait(&sm.s_full[wg], t & 1, abort_flag, P.status) &&
+           mbar_wait(&sm.q_full[slot], (t / NS) & 1, abort_flag, P.status);
+      if (ok && t > 0) ok = mbar_wait(&sm.pt_empty[wg], (t - 1) & 1, abort_flag, P.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      ++sc;
       tc_fence_after();
-      const bool msk = (P.causal && it == j) || ((it + 1) * kTile > P.N) || !key_ok;
+      const int row0 = it * kTile + wg * kHalf;
+      const bool msk = (P.causal && it == j) || (row0 + kHalf > P.N) || !key_ok;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t rs[32], rp[32];
-        tmem_ld32x2(t_lane + kColS + ch * 32, rs, t_lane + kColDP + ch * 32, rp);
-        if (ch == 3) {
+        tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
+        if (ch == 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_empty);
+          if (lane == 0) mbar_arrive(&sm.s_empty[wg]);
         }
         uint32_t wp[16], wd[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float4 tv = *reinterpret_cast<const float4*>(&sm.tau[slot][ch * 32 + e]);
-          const float4 dv = *reinterpret_cast<const float4*>(&sm.delta[slot][ch * 32 + e]);
+          const int r4 = wg * kHalf + ch * 32 + e;
+          const float4 tv = *reinterpret_cast<const float4*>(&sm.tau[slot][r4]);
+          const float4 dv = *reinterpret_cast<const float4*>(&sm.delta[slot][r4]);
           const float taus[4] = {tv.x, tv.y, tv.z, tv.w};
           const float dels[4] = {dv.x, dv.y, dv.z, dv.w};
           float pp[4], dd[4];
@@ -665,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < 4; ++u) {
             float tt = fmaf(__uint_as_float(rs[e + u]), P.c, -taus[u]);
             if (msk) {
-              const int row = it * kTile + ch * 32 + e + u;
+              const int row = row0 + ch * 32 + e + u;
               const bool ok_e = key_ok && row < P.N && (!P.causal || key <= row);
               if (!ok_e) tt = -1.0f;
             }
@@ -694,42 +723,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.pt_full);
-      ++ac;
+      if (lane == 0) mbar_arrive(&sm.pt_full[wg]);
     }
     if (ok && n > 0) {
       ok = mbar_wait(&sm.acc_full, 0, abort_flag, P.status);
       ok = __all_sync(0xffffffffu, ok);
     }
     tc_fence_after();
-    const size_t base = (static_cast<size_t>(bh) * P.N + key) * D;
+    // warpgroup 0 stores dV, warpgroup 1 stores dK
+    const uint32_t col = wg == 0 ? kColDV : kColDK;
+    const float scale = wg == 0 ? 1.0f : P.inv_sqrt_d;
+    __nv_bfloat16* dst_row = (wg == 0 ? P.dv : P.dk) + (static_cast<size_t>(bh) * P.N + key) * D;
 #pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t col = which == 0 ? kColDV : kColDK;
-      const float scale = which == 0 ? 1.0f : P.inv_sqrt_d;
-      __nv_bfloat16* dst_row = (which == 0 ? P.dv : P.dk) + base;
-#pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t r[32];
-        if (ok && n > 0) {
-          tmem_ld32(t_lane + col + ch * 32, r);
-        } else {
+    for (int ch = 0; ch < D / 32; ++ch) {
+      uint32_t r[32];
+      if (ok && n > 0) {
+        tmem_ld32(t_lane + col + ch * 32, r);
+      } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        for (int e = 0; e < 32; ++e) r[e] = 0u;
+      }
+      if (key_ok) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * scale,
+                                                          __uint_as_float(r[2 * e + 1]) * scale);
+          w[e] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        if (key_ok) {
-          uint32_t w[16];
+        uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 32);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * scale,
-                                                            __uint_as_float(r[2 * e + 1]) * scale);
-            w[e] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 32);
-#pragma unroll
-          for (int qd = 0; qd < 4; ++qd)
-            dst[qd] = make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
-        }
+        for (int qd = 0; qd < 4; ++qd)
+          dst[qd] = make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
       }
     }
     tc_fence_before();

@@ -145,7 +145,7 @@ int launch_bwd_row(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   static bool attr_ok = set_smem(kern, smem);
   if (!attr_ok) return ENTMAX_E_CUDA;
   const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.T);
-  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, p);
+  kern<<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
 }
 
@@ -158,7 +158,7 @@ int launch_bwd_col(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   static bool attr_ok = set_smem(kern, smem);
   if (!attr_ok) return ENTMAX_E_CUDA;
   const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.T);
-  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, p);
+  kern<<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
 }
 

@@ -158,12 +158,15 @@ struct FwdSmem {
   __nv_bfloat16 q[kTile * D];       // D/64 swizzled slabs
   __nv_bfloat16 k[NS][kTile * D];
   __nv_bfloat16 v[NS][kTile * D];
-  __nv_bfloat16 p[kTile * kTile];   // P tile, K-major (K = keys), 2 slabs
+  // P tiles, K-major (K = keys), 2 slabs each; double-buffered when D = 64
+  // leaves room, so the epilogue writes P(t+1) while the tensor core reads P(t)
+  static constexpr int kNSP = D == 64 ? 2 : 1;
+  __nv_bfloat16 p[kNSP][kTile * kTile];
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS];
   uint64_t v_full[NS], v_empty[NS];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full, p_empty, o_full, drain;
+  uint64_t p_full[kNSP], p_empty[kNSP], o_full, drain;
   uint32_t tmem_base;
   int abort_flag;
   int ctl_kind, ctl_n, ctl_iter;
@@ -182,7 +185,7 @@ constexpr int kMaxPrunes = 2;
 
 template <int D, int NS>
 __host__ __device__ constexpr int fwd_cand_cap() {
-  return (NS * kTile * D * 2 + kTile * kTile * 2) / (4 * kTile);
+  return (NS * kTile * D * 2 + FwdSmem<D, NS>::kNSP * kTile * kTile * 2) / (4 * kTile);
 }
 
 template <int D, int NS>
@@ -227,8 +230,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.s_empty[s], 4);
     }
-    mbar_init(&sm.p_full, 4);
-    mbar_init(&sm.p_empty, 1);
+    for (int s = 0; s < FwdSmem<D, NS>::kNSP; ++s) {
+      mbar_init(&sm.p_full[s], 4);
+      mbar_init(&sm.p_empty[s], 1);
+    }
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -396,11 +401,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         auto issue_pv = [&]() -> bool {
-          if (!mbar_wait(&sm.p_full, pc & 1, abort_flag, P.status)) return false;
+          constexpr uint32_t kNSP = FwdSmem<D, NS>::kNSP;
+          const uint32_t pb = pc % kNSP;
+          if (!mbar_wait(&sm.p_full[pb], (pc / kNSP) & 1, abort_flag, P.status)) return false;
           const uint32_t slot = vc % NS;
           if (!mbar_wait(&sm.v_full[slot], (vc / NS) & 1, abort_flag, P.status)) return false;
           tc_fence_after();
-          const uint32_t p_addr = smem_u32(sm.p);
+          const uint32_t p_addr = smem_u32(sm.p[pb]);
           const uint32_t v_addr = smem_u32(sm.v[slot]);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk) {
@@ -411,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        (pc > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&sm.v_empty[slot]);
-          mma_commit(&sm.p_empty);
+          mma_commit(&sm.p_empty[pb]);
           ++vc;
           ++pc;
           return true;
@@ -486,13 +493,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               // 9 bins in 7-bit lanes of one 64-bit word (<= 32 counts per chunk):
               // bin b of a score is floor(kNB * s) - (gtop - kNB), exact via a
               // round-down FMA against 1.5 * 2^23.
-              uint64_t packed = 0;
+              // four independent partial words (a single accumulator would chain
+              // 32 dependent 64-bit adds); lanes still hold at most 32 counts
+              uint64_t pk[4] = {0, 0, 0, 0};
 #pragma unroll
               for (int e = 0; e < 32; ++e) {
                 const float u = __fmaf_rd(fmaxf(v[e], vclamp), P.cN, kMagic);
                 const uint32_t sh = __float_as_uint(u) * 7u + cbase;
-                packed += shl64(1ull, sh);
+                pk[e & 3] += shl64(1ull, sh);
               }
+              const uint64_t packed = (pk[0] + pk[1]) + (pk[2] + pk[3]);
 #pragma unroll
               for (int b = 0; b <= kNB; ++b)
                 cnt[b] += static_cast<uint32_t>(packed >> (7 * b)) & 127u;
@@ -617,14 +627,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           Tmin = fminf(Tmin, fminf(fminf(tmin[0], tmin[1]), fminf(tmin[2], tmin[3])));
           Tneg = fmaxf(Tneg, fmaxf(fmaxf(tneg[0], tneg[1]), fmaxf(tneg[2], tneg[3])));
         } else {  // PASS_PV
+          constexpr uint32_t kNSP = FwdSmem<D, NS>::kNSP;
           const uint32_t cur_p = pc++;
-          if (cur_p > 0) {
-            ok = mbar_wait(&sm.p_empty, (cur_p - 1) & 1, abort_flag, P.status);
+          const uint32_t pb = cur_p % kNSP, puse = cur_p / kNSP;
+          if (puse > 0) {
+            ok = mbar_wait(&sm.p_empty[pb], (puse - 1) & 1, abort_flag, P.status);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
           }
           float part_lo = 0.f, part_hi = 0.f;
-          uint8_t* p_base = reinterpret_cast<uint8_t*>(sm.p);
+          uint8_t* p_base = reinterpret_cast<uint8_t*>(sm.p[pb]);
 #pragma unroll 1
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t r[32];
@@ -660,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.p_full);
+          if (lane == 0) mbar_arrive(&sm.p_full[pb]);
           rowsum += part_lo + part_hi;
           const uint32_t b_lo = __ballot_sync(0xffffffffu, row_ok && part_lo > 0.f);
           const uint32_t b_hi = __ballot_sync(0xffffffffu, row_ok && part_hi > 0.f);

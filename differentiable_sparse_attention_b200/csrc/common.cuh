@@ -47,14 +47,15 @@ __device__ __forceinline__ uint64_t shl64(uint64_t x, uint32_t sh) {
   return r;
 }
 
-// Offset (in 128-element rows) of the tile-max record of (row tile i, key tile
-// j) of head bh.  Causal problems store only the lower triangle j <= i.
+// Offset (in elements) of the tile-max record of (row tile i, key tile j) of
+// head bh: two halves (key columns 0-63 and 64-127) of 128 rows each.  Causal
+// problems store only the lower triangle j <= i.
 __device__ __forceinline__ size_t tmax_index(int bh, int i, int j, int tr, int tc, int causal) {
   const size_t per = causal ? static_cast<size_t>(tr) * (tr + 1) / 2
                             : static_cast<size_t>(tr) * tc;
   const size_t idx = causal ? static_cast<size_t>(i) * (i + 1) / 2 + j
                             : static_cast<size_t>(i) * tc + j;
-  return (static_cast<size_t>(bh) * per + idx) * kTile;
+  return (static_cast<size_t>(bh) * per + idx) * (2 * kTile);
 }
 
 // Byte offset, inside a 128-byte-swizzled K-major tile made of [128 rows][64

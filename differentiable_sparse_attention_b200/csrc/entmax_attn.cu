@@ -41,7 +41,7 @@ WsLayout ws_layout(int B, int H, int N, int D, int causal) {
   const size_t words = (t + 31) / 32;
   size_t off = 256;
   L.tmax = off;
-  off = align256(off + bh * tiles * kTile * sizeof(__half));
+  off = align256(off + bh * tiles * 2 * kTile * sizeof(__half));
   L.tilemask = off;
   off = align256(off + bh * t * words * sizeof(uint32_t));
   L.tilemaskT = off;
@@ -132,7 +132,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   static bool attr_ok = set_smem(kern, smem);
   if (!attr_ok) return ENTMAX_E_CUDA;
   const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.tr);
-  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  kern<<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
 }
 

@@ -1,24 +1,31 @@
 // Forward alpha-entmax attention kernel for sm_100a (bf16 inputs, f32 accumulate).
 //
-// One CTA owns a 128-row query tile of one (batch, head).  Warp 0 streams
-// K/V tiles with TMA, warp 1 issues tcgen05 MMAs into TMEM, warps 2-5 (one
-// thread per query row) run the epilogues.  The CTA walks a sequence of passes
-// over key tiles, each pass driven by a tile list in shared memory:
+// One CTA owns a 128-row query tile of one (batch, head).  Warp 0 streams K/V
+// tiles with TMA, warp 1 issues tcgen05 MMAs into TMEM, and warps 2-9 run the
+// epilogues as two warpgroups: warpgroup h handles key columns [64 h, 64 h + 64)
+// of every 128-key tile for all 128 query rows (one thread per row), keeps
+// its own half of the row's state, and the halves are merged in shared memory
+// at the end of each pass.  The CTA walks a sequence of passes over key tiles,
+// each driven by a tile list in shared memory:
 //
 //   HIST    every visible key tile: S = Q K^T, running row max, 8-bin
 //           histogram of the scores in the unit window below the max
-//           (AdaSplash-2 zh §2.1 / it §2A / ja §2.1 / es §2A), and a rounded-up
-//           per-(row, tile) score maximum kept in the workspace.  The reduced
-//           histogram problem gives tau_h with tau* - h <= tau_h <= tau*
-//           (Proposition 1 of the paper, as the summaries state it).
-//   REFINE  1..max_iter safeguarded steps from tau_h (zh §2.2, it §2B, ja §2.2,
-//           es §2B): Halley for alpha = 1.5, Newton for alpha = 2, bisection
-//           whenever the step leaves the bracket [lo, hi].  Only tiles whose
-//           recorded maximum exceeds the row's lower bound lo are visited:
-//           tiles entirely below lo <= tau* contribute nothing.
-//   PV      the surviving tiles: p = [s - tau]_+^(1/(alpha-1)) written to SMEM as
-//           bf16, O += P V on the tensor cores, and the bit-packed block mask
-//           (32 blocks per uint32 word, zh §2.3) of blocks holding a p > 0.
+//           (AdaSplash-2 zh §2.1 / it §2A / ja §2.1 / es §2A), the rounded-up
+//           per-(row, tile half) score maximum kept in the workspace, and the
+//           row's candidate scores (every score above a running lower bound of
+//           tau*).  The reduced histogram problem gives tau_h with
+//           tau* - h <= tau_h <= tau* (Proposition 1, as the summaries state it),
+//           and the safeguarded Halley (alpha = 1.5) / Newton (alpha = 2) steps
+//           (zh §2.2, it §2B, ja §2.2, es §2B) then run in registers over the
+//           candidates until the threshold is certified exact.
+//   COLLECT (only if a candidate list overflowed) rebuilds the lists above the
+//           final lower bound.
+//   REFINE  (only if a rebuilt list still overflows) refinement steps that
+//           stream the key tiles again.
+//   PV      tiles whose recorded maximum exceeds the row's lower bound:
+//           p = [s - tau]_+^(1/(alpha-1)) written to SMEM as bf16, O += P V on the
+//           tensor cores, and the bit-packed block mask (32 blocks per uint32
+//           word, zh §2.3) of blocks holding a p > 0.
 #pragma once
 
 #include <cstddef>
@@ -153,13 +160,29 @@ __device__ __forceinline__ bool solver_step(double F0, double F1, double F2, flo
   return exact;
 }
 
+constexpr int kFwdThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+
+__device__ __forceinline__ void fwd_epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Per-row state that warpgroup 1 hands to warpgroup 0 at the end of a pass.
+struct FwdXrow {
+  float m_raw;
+  int gtop;
+  int gtop_set;
+  float acc;
+  int ncand;
+  int over;
+  uint32_t cnt[kNB + 1];
+  float pad;
+};
+
 template <int D, int NS>
 struct FwdSmem {
   __nv_bfloat16 q[kTile * D];       // D/64 swizzled slabs
   __nv_bfloat16 k[NS][kTile * D];
   __nv_bfloat16 v[NS][kTile * D];
-  // P tiles, K-major (K = keys), 2 slabs each; double-buffered when D = 64
-  // leaves room, so the epilogue writes P(t+1) while the tensor core reads P(t)
+  // P tiles, K-major (K = keys), 2 slabs each (slab h written by warpgroup h);
+  // double-buffered when D = 64 leaves room
   static constexpr int kNSP = D == 64 ? 2 : 1;
   __nv_bfloat16 p[kNSP][kTile * kTile];
   uint64_t q_full;
@@ -175,13 +198,21 @@ struct FwdSmem {
   uint32_t flags[kMaxTiles / 32];
   uint32_t maskw[2][kMaxMaskWords];
   uint16_t tiles[kMaxTiles];
+  // warpgroup exchange
+  FwdXrow x1[kTile];          // 1 -> 0: histogram / candidate state
+  double xf[3][kTile];        // 1 -> 0: refinement partial sums
+  float xtmin[kTile], xtneg[kTile], xsum[kTile];
+  double xlo[kTile];          // 0 -> 1: bracket lower bound
+  float xtau[kTile];          // 0 -> 1: current threshold
+  int xflag[kTile];           // 0 -> 1: list rebuilt by COLLECT
 };
 
-// Candidate scores live in the V ring and the P tile, which stay idle until
+// Candidate scores live in the V ring and the P tiles, which stay idle until
 // the P.V pass: slot-major [cap][128 rows] floats (thread r uses column r, so
-// appends and reads are free of bank conflicts).  A row compacts its list at
-// most kMaxPrunes times; after that its list is rebuilt by a COLLECT pass.
-constexpr int kMaxPrunes = 2;
+// appends and reads are free of bank conflicts); warpgroup h owns slots
+// [h cap/2, (h + 1) cap/2).  A list is compacted at most kMaxPrunes times;
+// after that it is rebuilt by a COLLECT pass.
+constexpr int kMaxPrunes = 8;
 
 template <int D, int NS>
 __host__ __device__ constexpr int fwd_cand_cap() {
@@ -198,18 +229,33 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
+// Counts of a histogram whose top bin is g_from, re-expressed for top bin g_to >= g_from.
+__device__ __forceinline__ uint32_t hist_shifted(const uint32_t (&c)[kNB + 1], int b, int d) {
+  const int src = b + d;
+  uint32_t r = 0u;
+#pragma unroll
+  for (int s = 0; s <= kNB; ++s) r = (s == src) ? c[s] : r;
+  return r;
+}
+
 template <int D, int NS, bool ALPHA2>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     entmax_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const FwdParams P) {
   extern __shared__ uint8_t smem_raw[];
-  FwdSmem<D, NS>& sm = *reinterpret_cast<FwdSmem<D, NS>*>(align1024(smem_raw));
+  using Smem = FwdSmem<D, NS>;
+  Smem& sm = *reinterpret_cast<Smem*>(align1024(smem_raw));
   constexpr int kSlabs = D / 64;
   constexpr uint32_t kTileBytes = kTile * D * 2;
   constexpr uint32_t kIdescS = make_idesc(kTile, kTile, 1, 1, 0, 0);  // Q (K-major) x K (K-major)
   constexpr uint32_t kIdescPV = make_idesc(kTile, D, 1, 1, 0, 1);     // P (K-major) x V (MN-major)
   constexpr uint32_t kColO = 256;                                     // TMEM: S0, S1, O
+  constexpr uint32_t kNSP = Smem::kNSP;
+  constexpr int kCap = fwd_cand_cap<D, NS>();
+  constexpr int kCapH = kCap / 2;
+  static_assert(offsetof(Smem, p) == offsetof(Smem, v) + NS * kTile * D * 2,
+                "candidates need the V ring and the P tiles to be adjacent");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -228,10 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_empty[s], 4);
+      mbar_init(&sm.s_empty[s], 8);
     }
-    for (int s = 0; s < FwdSmem<D, NS>::kNSP; ++s) {
-      mbar_init(&sm.p_full[s], 4);
+    for (int s = 0; s < static_cast<int>(kNSP); ++s) {
+      mbar_init(&sm.p_full[s], 8);
       mbar_init(&sm.p_empty[s], 1);
     }
     mbar_init(&sm.o_full, 1);
@@ -244,9 +290,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.ctl_iter = 0;
     fence_mbar_init();
   }
-  for (int w = threadIdx.x; w < kMaxTiles / 32; w += kThreads) sm.flags[w] = 0u;
-  for (int w = threadIdx.x; w < 2 * kMaxMaskWords; w += kThreads) (&sm.maskw[0][0])[w] = 0u;
-  for (int t = threadIdx.x; t < ntc; t += kThreads) sm.tiles[t] = static_cast<uint16_t>(t);
+  for (int w = threadIdx.x; w < kMaxTiles / 32; w += kFwdThreads) sm.flags[w] = 0u;
+  for (int w = threadIdx.x; w < 2 * kMaxMaskWords; w += kFwdThreads) (&sm.maskw[0][0])[w] = 0u;
+  for (int t = threadIdx.x; t < ntc; t += kFwdThreads) sm.tiles[t] = static_cast<uint16_t>(t);
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
@@ -266,14 +312,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t kc = 0, vc = 0, sc = 0, pc = 0;   // K loads, V loads, S tiles, PV tiles
   bool q_issued = false, q_waited = false;
 
-  // epilogue (one query row per thread)
+  // epilogue: warpgroup wg, one query row per thread, key columns [hc0, hc0 + 64)
+  const int wg = warp >= 2 ? (warp - 2) >> 2 : 0;
+  const int hc0 = wg * 64;
   const int quad = warp & 3;
   const int rl = quad * 32 + lane;
   const int row = i * kTile + rl;
   const bool row_ok = (warp >= 2) && row < P.N;
   const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
   const int n_valid = P.causal ? min(row + 1, P.N) : P.N;
-  float m_raw = -INFINITY;                 // running max of q.k (raw units)
+  float m_raw = -INFINITY;                 // running max of q.k (raw units), this half
   int gtop = 0;                            // grid index floor(kNB * s) of the max
   bool gtop_set = false;
   uint32_t cnt[kNB + 1];
@@ -281,20 +329,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int b = 0; b <= kNB; ++b) cnt[b] = 0u;
   float vclamp = -P.slim;                  // scores are clamped to >= vclamp before binning
   uint32_t cbase = 0u;
-  // Candidate scores of this row: every q.k above acc_raw, which only grows and
-  // always stays at or below a lower bound of tau* (c * acc_raw <= tau*): the
-  // running max minus 1/c, raised to a partial-histogram tau_h when the list
-  // fills up and is pruned.  Scores left out are never in the support.
-  constexpr int kCap = fwd_cand_cap<D, NS>();
-  using Smem = FwdSmem<D, NS>;
-  static_assert(offsetof(Smem, p) == offsetof(Smem, v) + NS * kTile * D * 2,
-                "candidates need the V ring and the P tile to be adjacent");
-  float* my_cand = reinterpret_cast<float*>(&sm.v[0][0]) + rl;   // slot a at my_cand[a * 128]
+  // Candidate scores of this half of the row: every q.k above acc_raw, which
+  // only grows and always stays at or below a lower bound of tau* (the running
+  // max - 1/c, raised to the partial histogram's tau_h).  Scores left out are
+  // never in the support.
+  float* cand_base = reinterpret_cast<float*>(&sm.v[0][0]);
+  float* my_cand = cand_base + (wg * kCapH) * kTile + rl;     // slot a at my_cand[a * 128]
+  float* other_cand = cand_base + kCapH * kTile + rl;         // warpgroup 1's slots (read by 0)
   int ncand = 0;
   float acc_raw = -INFINITY;
   bool cand_over = false;
-  int prunes = 0;                          // list compactions so far (at most kMaxPrunes)
+  int prunes = 0;
   bool collect = false;                    // list rebuilt by a COLLECT pass above lo
+  int ncand1 = 0;                          // warpgroup 0: size of warpgroup 1's list
   double lo = 0.0, hi = 0.0;               // bracket of tau*
   double l_drop = -INFINITY;               // every score left out of the candidates is <= l_drop
   float tau_c = 0.0f;                      // current evaluation point / final tau
@@ -303,19 +350,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   float rowsum = 0.0f;
 
   auto trace_store = [&](int it, float val) {
-    if (P.tau_trace != nullptr && row_ok && it <= P.max_iter)
+    if (P.tau_trace != nullptr && row_ok && wg == 0 && it <= P.max_iter)
       P.tau_trace[(static_cast<size_t>(it) * P.BH + bh) * P.N + row] = val;
   };
-
-  // Per-element validity only matters on the diagonal tile (causal) and on
-  // the ragged last key tile.
   auto needs_mask = [&](int j) {
-    return (P.causal && j == i) || ((j + 1) * kTile > P.N);
+    return (P.causal && j == i) || (j * kTile + hc0 + 64 > P.N);
   };
   auto apply_mask = [&](float (&v)[32], int j, int ch) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-      const int col = j * kTile + ch * 32 + e;
+      const int col = j * kTile + hc0 + ch * 32 + e;
       const bool ok = col < P.N && (!P.causal || col <= row);
       v[e] = ok ? v[e] : -INFINITY;
     }
@@ -401,7 +445,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         auto issue_pv = [&]() -> bool {
-          constexpr uint32_t kNSP = FwdSmem<D, NS>::kNSP;
           const uint32_t pb = pc % kNSP;
           if (!mbar_wait(&sm.p_full[pb], (pc / kNSP) & 1, abort_flag, P.status)) return false;
           const uint32_t slot = vc % NS;
@@ -439,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       // ------------------------------------------------------------ epilogue
       bool ok = true;
-      double F0 = 0.0, F1 = 0.0, F2 = 0.0;  // refinement sums at tau_c
+      double F0 = 0.0, F1 = 0.0, F2 = 0.0;  // refinement sums at tau_c (this half)
       float Tmin = INFINITY;                // smallest positive s - tau_c
       float Tneg = -INFINITY;               // largest non-positive s - tau_c
       if (kind == PASS_PV) rowsum = 0.0f;
@@ -452,13 +495,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const bool msk = needs_mask(j);
-        const uint32_t t_s = t_lane + sb * kTile;
+        const uint32_t t_s = t_lane + sb * kTile + hc0;
 
         if (kind == PASS_HIST) {
           float tile_max = -INFINITY;
-          float cmx0 = -INFINITY, cmx1 = -INFINITY, cmx2 = -INFINITY, cmx3 = -INFINITY;
+          float cmx0 = -INFINITY, cmx1 = -INFINITY;
 #pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
+          for (int ch = 0; ch < 2; ++ch) {
             uint32_t r[32];
             tmem_ld32(t_s + ch * 32, r);
             float v[32];
@@ -490,11 +533,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 vclamp = (static_cast<float>(gtop - kNB) - 1.5f) / P.cN;
                 cbase = 0u - 7u * (kMagicBits + static_cast<uint32_t>(gtop - kNB));
               }
-              // 9 bins in 7-bit lanes of one 64-bit word (<= 32 counts per chunk):
-              // bin b of a score is floor(kNB * s) - (gtop - kNB), exact via a
-              // round-down FMA against 1.5 * 2^23.
-              // four independent partial words (a single accumulator would chain
-              // 32 dependent 64-bit adds); lanes still hold at most 32 counts
+            }
+            // A chunk whose maximum lies below the window adds nothing to the
+            // histogram (common once the running max has settled): skip it.
+            if (cm > vclamp) {
+              // 9 bins in 7-bit lanes of 64-bit words: bin b of a score is
+              // floor(kNB * s) - (gtop - kNB), exact via a round-down FMA against
+              // 1.5 * 2^23; four independent words (one would chain 32 dependent
+              // 64-bit adds), lanes hold at most 32 counts.
               uint64_t pk[4] = {0, 0, 0, 0};
 #pragma unroll
               for (int e = 0; e < 32; ++e) {
@@ -508,25 +554,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cnt[b] += static_cast<uint32_t>(packed >> (7 * b)) & 127u;
             }
             if (ch == 0) cmx0 = cm;
-            else if (ch == 1) cmx1 = cm;
-            else if (ch == 2) cmx2 = cm;
-            else cmx3 = cm;
+            else cmx1 = cm;
           }
-          // Candidates of this tile: every score above acc_raw, a lower bound of
-          // tau* (the running max - 1, raised to the partial histogram's tau_h
-          // -- tau_h of the scores seen so far, this tile included -- whenever
-          // some chunk of the tile reaches the current bound).
+          // Candidates of this tile half: every score above acc_raw, raised to the
+          // partial histogram's tau_h (scores seen so far by this warpgroup)
+          // whenever a chunk reaches the current bound.
           {
-            const float cmt = fmaxf(fmaxf(cmx0, cmx1), fmaxf(cmx2, cmx3));
             acc_raw = fmaxf(acc_raw, __fsub_rd(m_raw, P.inv_c));
-            if (row_ok && !cand_over && gtop_set && cmt > acc_raw) {
+            if (row_ok && !cand_over && gtop_set && fmaxf(cmx0, cmx1) > acc_raw) {
               const double th = hist_threshold<ALPHA2>(cnt, gtop);
               acc_raw = fmaxf(acc_raw, __double2float_rd((th - hist_margin(th)) / P.c));
             }
           }
 #pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
-            const float cm = ch == 0 ? cmx0 : ch == 1 ? cmx1 : ch == 2 ? cmx2 : cmx3;
+          for (int ch = 0; ch < 2; ++ch) {
+            const float cm = ch == 0 ? cmx0 : cmx1;
             const bool want = row_ok && !cand_over && cm > acc_raw;
             if (!__any_sync(0xffffffffu, want)) continue;
             uint32_t r[32];
@@ -536,9 +578,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (msk) apply_mask(v, j, ch);
-            if (ncand + 32 > kCap) {
+            if (ncand + 32 > kCapH) {
               if (prunes < kMaxPrunes) {
-                // drop the listed scores that fell below the bound
                 ++prunes;
                 int kept = 0;
                 for (int a = 0; a < ncand; ++a) {
@@ -547,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ncand = kept;
               }
-              cand_over = ncand + 32 > kCap;
+              cand_over = ncand + 32 > kCapH;
             }
             if (!cand_over) {
 #pragma unroll
@@ -560,15 +601,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
           const float rec = row_ok ? tile_max * P.c : -INFINITY;
-          P.tmax[tmax_index(bh, i, j, P.tr, P.tc, P.causal) + rl] = __float2half_ru(rec);
+          P.tmax[tmax_index(bh, i, j, P.tr, P.tc, P.causal) + wg * kTile + rl] =
+              __float2half_ru(rec);
         } else if (kind == PASS_COLLECT) {
           // rebuild the lists of the rows that overflowed: exactly the scores above lo
           const float thr = collect ? __double2float_rd(lo / P.c) : INFINITY;
 #pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
+          for (int ch = 0; ch < 2; ++ch) {
             uint32_t r[32];
             tmem_ld32(t_s + ch * 32, r);
-            if (ch == 3) {
+            if (ch == 1) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
@@ -581,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               if (v[e] > thr) {
-                if (ncand < kCap) my_cand[ncand * kTile] = v[e];
+                if (ncand < kCapH) my_cand[ncand * kTile] = v[e];
                 ++ncand;
               }
             }
@@ -593,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float tmin[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
           float tneg[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
+          for (int ch = 0; ch < 2; ++ch) {
             uint32_t r[32];
             tmem_ld32(t_s + ch * 32, r);
             float v[32];
@@ -627,7 +669,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           Tmin = fminf(Tmin, fminf(fminf(tmin[0], tmin[1]), fminf(tmin[2], tmin[3])));
           Tneg = fmaxf(Tneg, fmaxf(fmaxf(tneg[0], tneg[1]), fmaxf(tneg[2], tneg[3])));
         } else {  // PASS_PV
-          constexpr uint32_t kNSP = FwdSmem<D, NS>::kNSP;
           const uint32_t cur_p = pc++;
           const uint32_t pb = cur_p % kNSP, puse = cur_p / kNSP;
           if (puse > 0) {
@@ -635,13 +676,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
           }
-          float part_lo = 0.f, part_hi = 0.f;
+          float part = 0.f;
           uint8_t* p_base = reinterpret_cast<uint8_t*>(sm.p[pb]);
 #pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
+          for (int ch = 0; ch < 2; ++ch) {
             uint32_t r[32];
             tmem_ld32(t_s + ch * 32, r);
-            if (ch == 3) {
+            if (ch == 1) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
@@ -662,34 +703,32 @@ __global__ void __launch_bounds__(kThreads, 1)
               const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
               w[e] = *reinterpret_cast<const uint32_t*>(&h2);
             }
-            const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-            if (ch < 2) part_lo += psum; else part_hi += psum;
+            part += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            // keys hc0 + 32 ch + 8 qd .. : slab wg of the K-major P tile
 #pragma unroll
             for (int qd = 0; qd < 4; ++qd) {
-              *reinterpret_cast<uint4*>(p_base + sw128_chunk_offset(rl, ch * 4 + qd)) =
+              *reinterpret_cast<uint4*>(p_base + sw128_chunk_offset(rl, wg * 8 + ch * 4 + qd)) =
                   make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
             }
           }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.p_full[pb]);
-          rowsum += part_lo + part_hi;
-          const uint32_t b_lo = __ballot_sync(0xffffffffu, row_ok && part_lo > 0.f);
-          const uint32_t b_hi = __ballot_sync(0xffffffffu, row_ok && part_hi > 0.f);
-          if (lane == 0) {
+          rowsum += part;
+          const uint32_t bits = __ballot_sync(0xffffffffu, row_ok && part > 0.f);
+          if (lane == 0 && bits != 0u) {
             if (P.block == kTile) {
-              if (b_lo | b_hi) atomicOr(&sm.maskw[0][j >> 5], 1u << (j & 31));
-            } else {  // block 64: two mask rows per tile, two key blocks per tile
+              atomicOr(&sm.maskw[0][j >> 5], 1u << (j & 31));
+            } else {  // block 64: two mask rows per tile, key block 2 j + wg
               const int h = quad >> 1;
-              const int kb = 2 * j;
-              if (b_lo) atomicOr(&sm.maskw[h][kb >> 5], 1u << (kb & 31));
-              if (b_hi) atomicOr(&sm.maskw[h][(kb + 1) >> 5], 1u << ((kb + 1) & 31));
+              const int kb = 2 * j + wg;
+              atomicOr(&sm.maskw[h][kb >> 5], 1u << (kb & 31));
             }
           }
         }
       }
 
-      // ---------------- end of pass: solver step and the next tile list
+      // ---------------- end of pass: merge the halves, solve, next tile list
       auto build_list = [&](double thr_d) {
         const float thr = row_ok ? __double2float_rd(thr_d) : INFINITY;
         for (int t = 0; t < n; t += 4) {
@@ -699,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < 4; ++u) {
             jj[u] = (t + u < n) ? static_cast<int>(sm.tiles[t + u]) : -1;
             hv[u] = jj[u] >= 0 ? __half2float(P.tmax[tmax_index(bh, i, jj[u], P.tr, P.tc,
-                                                                 P.causal) + rl])
+                                                                 P.causal) + wg * kTile + rl])
                                : -INFINITY;
           }
 #pragma unroll
@@ -710,23 +749,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
-
-      // Refinement over the row's candidate list (every score that can be in
-      // the support), in registers: no further pass over the keys.
+      // Refinement over the row's candidate lists (warpgroup 0: both halves), in
+      // registers, once the lists hold every score above lo.
       auto refine_registers = [&]() {
-        // only once the list holds every score above lo: after HIST for rows
-        // whose list never overflowed, after COLLECT for the rebuilt ones
-        if (!row_ok || cand_over || (collect && kind == PASS_HIST)) return;
+        if (wg != 0 || !row_ok || cand_over || (collect && kind == PASS_HIST)) return;
         for (; iter < P.max_iter && !row_done;) {
           float f0[4] = {0.f, 0.f, 0.f, 0.f}, f1[4] = {0.f, 0.f, 0.f, 0.f},
                 f2[4] = {0.f, 0.f, 0.f, 0.f};
           float tmn[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
           float tng[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          for (int e0 = 0; e0 < ncand; e0 += 4) {
+          const int ntot = ncand + ncand1;
+          for (int e0 = 0; e0 < ntot; e0 += 4) {
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
-              const float tt =
-                  e0 + a < ncand ? fmaf(my_cand[(e0 + a) * kTile], P.c, -tau_c) : -INFINITY;
+              const int e = e0 + a;
+              float tt = -INFINITY;
+              if (e < ncand) tt = fmaf(my_cand[e * kTile], P.c, -tau_c);
+              else if (e < ntot) tt = fmaf(other_cand[(e - ncand) * kTile], P.c, -tau_c);
               const bool in = tt > 0.0f;
               const float tp = fmaxf(tt, 0.0f);
               tmn[a] = in ? fminf(tmn[a], tt) : tmn[a];
@@ -751,6 +790,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           trace_store(iter, tau_c);
         }
       };
+      // warpgroup 0 -> 1: the row's threshold, lower bound and COLLECT flag
+      auto publish = [&]() {
+        if (wg == 0) {
+          sm.xtau[rl] = tau_c;
+          sm.xlo[rl] = lo;
+          sm.xflag[rl] = collect ? 1 : 0;
+        }
+        fwd_epi_bar();
+        if (wg == 1) {
+          tau_c = sm.xtau[rl];
+          lo = sm.xlo[rl];
+          collect = sm.xflag[rl] != 0;
+        }
+      };
       // Publish the next pass: PV unless some row still needs its list rebuilt
       // (COLLECT) or must refine over the key tiles (REFINE).
       auto next_pass = [&](int passes_done_kind) {
@@ -758,7 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tensor core use next: order these generic accesses before them
         fence_proxy_async_smem();
         build_list(lo);
-        epi_bar();
+        fwd_epi_bar();
         if (warp == 2) {
           const int nn = compact_tiles(sm.flags, (ntc + 31) >> 5, sm.tiles);
           if (lane == 0) {
@@ -776,8 +829,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       if (kind == PASS_HIST) {
+        if (wg == 1) {
+          FwdXrow& x = sm.x1[rl];
+          x.m_raw = m_raw;
+          x.gtop = gtop;
+          x.gtop_set = gtop_set ? 1 : 0;
+          x.acc = acc_raw;
+          x.ncand = ncand;
+          x.over = cand_over ? 1 : 0;
+#pragma unroll
+          for (int b = 0; b <= kNB; ++b) x.cnt[b] = cnt[b];
+        }
+        fwd_epi_bar();
         double tau_h = 0.0;
-        if (row_ok) {
+        if (wg == 0 && row_ok) {
+          // merge warpgroup 1's half of the row into this one
+          const FwdXrow& x = sm.x1[rl];
+          if (x.gtop_set) {
+            uint32_t c1[kNB + 1];
+#pragma unroll
+            for (int b = 0; b <= kNB; ++b) c1[b] = x.cnt[b];
+            const int g = gtop_set ? max(gtop, x.gtop) : x.gtop;
+            const int d0 = gtop_set ? g - gtop : kNB + 1;
+            const int d1 = g - x.gtop;
+#pragma unroll
+            for (int b = 0; b <= kNB; ++b) {
+              const uint32_t a0 = d0 <= kNB ? hist_shifted(cnt, b, d0) : 0u;
+              const uint32_t a1 = d1 <= kNB ? hist_shifted(c1, b, d1) : 0u;
+              cnt[b] = a0 + a1;
+            }
+            gtop = g;
+            gtop_set = true;
+          }
+          m_raw = fmaxf(m_raw, x.m_raw);
+          acc_raw = fmaxf(acc_raw, x.acc);
+          ncand1 = x.ncand;
+          cand_over = cand_over || x.over;
           if (fabsf(m_raw * P.cN) >= 2097152.0f) atomicOr(P.status, ST_RANGE);
           tau_h = hist_threshold<ALPHA2>(cnt, gtop);
           const double margin = hist_margin(tau_h);
@@ -791,40 +878,61 @@ __global__ void __launch_bounds__(kThreads, 1)
           tau_c = __double2float_rd(lo);
           lo = tau_c;
           if (cand_over && P.max_iter > 0) {
-            // the list lost scores: rebuild it above lo in a COLLECT pass
+            // a list lost scores: rebuild both halves above lo in a COLLECT pass
             collect = true;
             cand_over = false;
-            ncand = 0;
             l_drop = lo;
             sm.cand_overflow = 1;
           }
         }
         iter = 0;
         trace_store(0, static_cast<float>(tau_h));
-        epi_bar();
         refine_registers();
+        publish();
+        if (collect) {
+          ncand = 0;
+          cand_over = false;
+        }
         next_pass(CNT_HIST_TILES);
         if (warp == 2 && lane == 0 && sm.ctl_kind == PASS_COLLECT)
           atomicAdd(&P.counters[CNT_CAND_OVERFLOW], 1ull);
       } else if (kind == PASS_COLLECT) {
-        if (row_ok && collect) {
-          cand_over = ncand > kCap;
+        if (wg == 1) sm.x1[rl].ncand = ncand;
+        fwd_epi_bar();
+        if (wg == 0 && row_ok && collect) {
+          ncand1 = sm.x1[rl].ncand;
+          cand_over = ncand > kCapH || ncand1 > kCapH;
           if (cand_over) sm.cand_overflow = 2;   // refine this tile over the key tiles
         }
-        epi_bar();
+        fwd_epi_bar();
         if (warp == 2 && lane == 0 && sm.cand_overflow == 1) sm.cand_overflow = 0;
-        epi_bar();
+        fwd_epi_bar();
         refine_registers();
-        if (row_ok && !row_done && iter < P.max_iter) sm.not_converged = 1;
+        if (wg == 0 && row_ok && !row_done && iter < P.max_iter) sm.not_converged = 1;
+        publish();
         next_pass(CNT_REFINE_TILES);
       } else if (kind == PASS_REFINE) {
-        if (row_ok && !row_done && iter < P.max_iter) {
+        if (wg == 1) {
+          sm.xf[0][rl] = F0;
+          sm.xf[1][rl] = F1;
+          sm.xf[2][rl] = F2;
+          sm.xtmin[rl] = Tmin;
+          sm.xtneg[rl] = Tneg;
+        }
+        fwd_epi_bar();
+        if (wg == 0 && row_ok && !row_done && iter < P.max_iter) {
+          F0 += sm.xf[0][rl];
+          F1 += sm.xf[1][rl];
+          F2 += sm.xf[2][rl];
+          Tmin = fminf(Tmin, sm.xtmin[rl]);
+          Tneg = fmaxf(Tneg, sm.xtneg[rl]);
           row_done = solver_step<ALPHA2>(F0, F1, F2, Tmin, Tneg, l_drop, tau_c, lo, hi);
           ++iter;
           trace_store(iter, tau_c);
           if (!row_done && iter < P.max_iter) sm.not_converged = 1;
         }
         if (warp == 2 && lane == 0) ++sm.ctl_iter;
+        publish();
         next_pass(CNT_REFINE_TILES);
       } else {  // PASS_PV: write O, tau, mask
         if (ok && n > 0) {
@@ -833,8 +941,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         __nv_bfloat16* orow = P.out + (static_cast<size_t>(bh) * P.N + row) * D;
+        // warpgroup wg stores O columns [wg D/2, (wg + 1) D/2)
 #pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int ch = wg * (D / 64); ch < (wg + 1) * (D / 64); ++ch) {
           uint32_t r[32];
           if (ok && n > 0) {
             tmem_ld32(t_lane + kColO + ch * 32, r);
@@ -856,16 +965,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               dst[qd] = make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
           }
         }
-        if (row_ok) {
+        if (wg == 1) sm.xsum[rl] = rowsum;
+        tc_fence_before();
+        fwd_epi_bar();
+        if (wg == 0 && row_ok) {
+          rowsum += sm.xsum[rl];
           P.tau[static_cast<size_t>(bh) * P.N + row] = tau_c;
           if (!(fabsf(rowsum - 1.0f) <= 1e-3f)) atomicOr(P.status, ST_NOT_CONVERGED);
         }
-        for (int it = iter + 1; it <= P.max_iter; ++it) trace_store(it, tau_c);
-        tc_fence_before();
-        epi_bar();
+        if (wg == 0)
+          for (int it = iter + 1; it <= P.max_iter; ++it) trace_store(it, tau_c);
         const int spr = kTile / P.block;
         const int et = threadIdx.x - 64;
-        for (int idx = et; idx < spr * P.mask_words; idx += kEpiThreads) {
+        for (int idx = et; idx < spr * P.mask_words; idx += kFwdThreads - 64) {
           const int h = idx / P.mask_words;
           const int w = idx - h * P.mask_words;
           const int mrow = i * spr + h;

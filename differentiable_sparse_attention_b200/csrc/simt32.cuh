@@ -163,15 +163,17 @@ __global__ void __launch_bounds__(128) entmax_fwd_f32_kernel(const F32Params P) 
         vclamp = (static_cast<float>(gtop - kNB) - 1.5f) / P.cN;
         cbase = 0u - 7u * (kMagicBits + static_cast<uint32_t>(gtop - kNB));
       }
-      uint64_t pk[4] = {0, 0, 0, 0};
+      if (cm > vclamp) {   // a chunk entirely below the window adds nothing
+        uint64_t pk[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float u = __fmaf_rd(fmaxf(v[e], vclamp), P.cN, kMagic);
-        pk[e & 3] += shl64(1ull, __float_as_uint(u) * 7u + cbase);
+        for (int e = 0; e < 32; ++e) {
+          const float u = __fmaf_rd(fmaxf(v[e], vclamp), P.cN, kMagic);
+          pk[e & 3] += shl64(1ull, __float_as_uint(u) * 7u + cbase);
+        }
+        const uint64_t packed = (pk[0] + pk[1]) + (pk[2] + pk[3]);
+#pragma unroll
+        for (int b = 0; b <= kNB; ++b) cnt[b] += static_cast<uint32_t>(packed >> (7 * b)) & 127u;
       }
-      const uint64_t packed = (pk[0] + pk[1]) + (pk[2] + pk[3]);
-#pragma unroll
-      for (int b = 0; b <= kNB; ++b) cnt[b] += static_cast<uint32_t>(packed >> (7 * b)) & 127u;
       acc_raw = fmaxf(acc_raw, __fsub_rd(m_raw, P.inv_c));
       if (row_ok && !cand_over && cm > acc_raw) {
         const double th = hist_threshold<ALPHA2>(cnt, gtop);

@@ -140,8 +140,8 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
  * every GPU that loads the library holds those 8 MiB until the process exits.
  * The call allocates nothing and calls no allocating routine.
  *   - Problems whose scratch exceeds the 8 MiB return ENTMAX_E_SCRATCH and
- *     launch nothing (causal: 256 + B*H*T*(T+1)/2*256 bytes, T = ceil(N/128);
- *     e.g. B*H = 32 at N = 4096 needs 4.3 MB).
+ *     launch nothing (causal: 256 + B*H*T*(T+1)/2*512 bytes, T = ceil(N/128);
+ *     e.g. B*H = 16 at N = 4096 needs 4.3 MB).
  *   - The array's device address is looked up once per device, on the first
  *     call made while that device is current; make that first call before any
  *     stream capture on the device.

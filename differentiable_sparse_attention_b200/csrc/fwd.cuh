@@ -508,7 +508,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (msk) apply_mask(v, j, ch);
-            const float cm = max32(v);
+            // maxima of the four 8-score groups, then of the chunk (a tree)
+            float gm[4];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              float a = fmaxf(fmaxf(v[8 * g], v[8 * g + 1]), fmaxf(v[8 * g + 2], v[8 * g + 3]));
+              float b = fmaxf(fmaxf(v[8 * g + 4], v[8 * g + 5]), fmaxf(v[8 * g + 6], v[8 * g + 7]));
+              gm[g] = fmaxf(a, b);
+            }
+            const float cm = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
             tile_max = fmaxf(tile_max, cm);
             m_raw = fmaxf(m_raw, cm);
             if (cm > -INFINITY) {
@@ -536,19 +544,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             // A chunk whose maximum lies below the window adds nothing to the
             // histogram (common once the running max has settled): skip it.
+            // Only 8-score groups reaching the window add to the histogram (most
+            // scores of a long row lie far below it once the running max has
+            // settled).  9 bins in 7-bit lanes of 64-bit words: bin b of a score
+            // is floor(kNB * s) - (gtop - kNB), exact via a round-down FMA against
+            // 1.5 * 2^23; two independent words, lanes hold at most 32 counts.
             if (cm > vclamp) {
-              // 9 bins in 7-bit lanes of 64-bit words: bin b of a score is
-              // floor(kNB * s) - (gtop - kNB), exact via a round-down FMA against
-              // 1.5 * 2^23; four independent words (one would chain 32 dependent
-              // 64-bit adds), lanes hold at most 32 counts.
-              uint64_t pk[4] = {0, 0, 0, 0};
+              uint64_t pk0 = 0, pk1 = 0;
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const float u = __fmaf_rd(fmaxf(v[e], vclamp), P.cN, kMagic);
-                const uint32_t sh = __float_as_uint(u) * 7u + cbase;
-                pk[e & 3] += shl64(1ull, sh);
+              for (int g = 0; g < 4; ++g) {
+                if (gm[g] > vclamp) {
+#pragma unroll
+                  for (int e = 8 * g; e < 8 * g + 8; ++e) {
+                    const float u = __fmaf_rd(fmaxf(v[e], vclamp), P.cN, kMagic);
+                    const uint32_t sh = __float_as_uint(u) * 7u + cbase;
+                    if (e & 1) pk1 += shl64(1ull, sh);
+                    else pk0 += shl64(1ull, sh);
+                  }
+                }
               }
-              const uint64_t packed = (pk[0] + pk[1]) + (pk[2] + pk[3]);
+              const uint64_t packed = pk0 + pk1;
 #pragma unroll
               for (int b = 0; b <= kNB; ++b)
                 cnt[b] += static_cast<uint32_t>(packed >> (7 * b)) & 127u;
@@ -753,6 +768,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // registers, once the lists hold every score above lo.
       auto refine_registers = [&]() {
         if (wg != 0 || !row_ok || cand_over || (collect && kind == PASS_HIST)) return;
+        // keep only the candidates above lo (the others contribute nothing at any
+        // tau >= lo), so the iterations run over roughly the support
+        {
+          const float thr = __double2float_rd(lo / P.c);
+          int kept = 0;
+          for (int a = 0; a < ncand; ++a) {
+            const float xa = my_cand[a * kTile];
+            if (xa > thr) my_cand[(kept++) * kTile] = xa;
+          }
+          ncand = kept;
+          kept = 0;
+          for (int a = 0; a < ncand1; ++a) {
+            const float xa = other_cand[a * kTile];
+            if (xa > thr) other_cand[(kept++) * kTile] = xa;
+          }
+          ncand1 = kept;
+          l_drop = fmax(l_drop, static_cast<double>(thr) * P.c);
+        }
         for (; iter < P.max_iter && !row_done;) {
           float f0[4] = {0.f, 0.f, 0.f, 0.f}, f1[4] = {0.f, 0.f, 0.f, 0.f},
                 f2[4] = {0.f, 0.f, 0.f, 0.f};

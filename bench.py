@@ -215,8 +215,9 @@ def run_ours(args, points, rank, world, device):
             phase_tot[n] += phases[n]
         for n, v in cnt.items():
             counters_acc[n] = counters_acc.get(n, 0) + v
-        # our kernels per step: forward; 4 fp16 copies + 2 tile-mask kernels + row + column
-        kernel_launches += args.steps * (1 + 4 + 2 + 2)
+        # our kernels per step: forward (fp16 copy of v + kernel); backward (fp16 copies
+        # of q, k, dout + 2 tile-mask kernels + row + column)
+        kernel_launches += args.steps * (2 + 3 + 2 + 2)
 
         # ---- end to end through the public API: pinned host buffers in and out
         e2e = None
@@ -300,8 +301,9 @@ def merge_clocks(cl):
 def roofline_for(kernel, ms, points, results, peaks, peaks_kind, steps):
     """Achieved vs peak for the dominant kernel.  Tensor-bound kernels count the
     MMA FLOPs their tile lists imply (128 x 128 tiles):
-      forward:   (hist + refine tiles) * 2*128*128*D + pv tiles * 4*128*128*D
-      bwd row:   row tiles * (2 passes * 2 + 1) * 2*128*128*D   (S, dP twice; dQ)
+      forward:   (hist + refine tiles) * 2*128*128*D + pv tiles * 3 * 2*128*128*D
+                 (S, P.V, G.V)
+      bwd row:   row tiles * 3 * 2*128*128*D                    (S, dP, dQ)
       bwd col:   col tiles * 4 * 2*128*128*D                    (S^T, dP^T, dV, dK)
     """
     fl = 0.0
@@ -309,9 +311,9 @@ def roofline_for(kernel, ms, points, results, peaks, peaks_kind, steps):
         c = r["counters"]
         unit = 2.0 * 128 * 128 * w.D
         if kernel == "fwd":
-            fl += ((c["fwd_hist_tiles"] + c["fwd_refine_tiles"]) + 2 * c["fwd_pv_tiles"]) * unit
+            fl += ((c["fwd_hist_tiles"] + c["fwd_refine_tiles"]) + 3 * c["fwd_pv_tiles"]) * unit
         elif kernel == "bwd_row":
-            fl += c["bwd_row_tiles"] * 5 * unit
+            fl += c["bwd_row_tiles"] * 3 * unit
         elif kernel == "bwd_col":
             fl += c["bwd_col_tiles"] * 4 * unit
     fl /= len(points)

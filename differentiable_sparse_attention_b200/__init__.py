@@ -154,7 +154,11 @@ def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = True, block: int
 def entmax_attn_bwd(q, k, v, dout, tau, mask, alpha: float = 1.5, causal: bool = True,
                     block: int = 128, *, dq=None, dk=None, dv=None, workspace=None,
                     stream=None):
-    """alpha-entmax attention backward through ``entmax_attn_bwd``; returns (dq, dk, dv)."""
+    """alpha-entmax attention backward through ``entmax_attn_bwd``; returns (dq, dk, dv).
+
+    For bf16 inputs ``workspace`` must be the one the forward of the same
+    inputs wrote (``Forward.workspace``): it carries the forward's g-weighted
+    means of v and its fp16 copy of v."""
     _check_qkv(q, k, v, dout)
     B, H, N, D = q.shape
     dev = q.device
@@ -162,6 +166,8 @@ def entmax_attn_bwd(q, k, v, dout, tau, mask, alpha: float = 1.5, causal: bool =
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     if workspace is None:
+        if q.dtype == torch.bfloat16:
+            raise ValueError("entmax_attn_bwd: bf16 needs the forward's workspace")
         workspace = alloc_workspace(B, H, N, D, block, causal, dev)
     rc = _lib().entmax_attn_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(tau), _ptr(mask), B, H, N, D,

@@ -10,8 +10,9 @@
 //
 //   tile_mask_kernel / tile_mask_t_kernel  block mask -> 128x128 tile mask and its
 //                                          transpose (workspace)
-//   entmax_bwd_row_kernel   one CTA per 128-row query tile: pass A computes
-//                           delta over the active key tiles, pass B dQ.
+//   entmax_bwd_row_kernel   one CTA per 128-row query tile: delta from dO and
+//                           the forward's g-weighted means of v, then dQ in one
+//                           pass over the active key tiles.
 //   entmax_bwd_col_kernel   one CTA per 128-key tile: dK and dV over the active
 //                           query tiles, accumulated in TMEM (no atomics).
 #pragma once
@@ -107,6 +108,8 @@ struct BwdParams {
   const float* tau;          // [BH][N]
   const uint32_t* tm;        // tile mask rows (row kernel) or transposed rows (column kernel)
   float* delta;              // workspace [BH][N]
+  const float* vbar;         // [BH][N][D] g-weighted means of v from the forward
+  const __half* dout16;      // [BH][N][D] fp16 copy of dO
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
@@ -153,6 +156,9 @@ constexpr int kHalfBytes = kTile * kHalf * 2;   // one [128][64] fp16 slab
 __device__ __forceinline__ void bwd_epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // ============================================================ row kernel (delta, dQ)
+// delta_r = sum_c g dP / sum_c g with dP = dO V^T is dO_r . vbar_r, the dot of
+// the row's output gradient with the forward's g-weighted mean of v: the row
+// kernel forms it in its prologue and then runs a single pass over the tiles.
 template <int D, int NSK, int NSV>
 struct BwdRowSmem {
   __half q[kTile * D];
@@ -160,8 +166,7 @@ struct BwdRowSmem {
   __half k[NSK][kTile * D];
   __half v[NSV][kTile * D];
   __half ds[2][kTile * kHalf];       // dS half tiles [128 rows][64 keys], K-major
-  float part_gdp[2][kTile];          // pass-A partial sums per warpgroup
-  float part_g[2][kTile];
+  float part_delta[2][kTile];        // half-dot products per warpgroup
   uint64_t qdo_full;
   uint64_t k_full[NSK], k_empty[NSK];
   uint64_t v_full[NSV], v_empty[NSV];
@@ -183,7 +188,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_do, const BwdParams P) {
-  static_assert(NSK >= 2, "pass B keeps K(t-1) while S(t) is issued");
+  static_assert(NSK >= 2, "K(t - 1) stays for its dQ step while S(t) is issued");
   extern __shared__ uint8_t smem_raw[];
   auto& sm = *reinterpret_cast<BwdRowSmem<D, NSK, NSV>*>(align1024(smem_raw));
   constexpr int kSlabs = D / 64;
@@ -240,7 +245,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_3d(sm.q + s * kTile * 64, &tm_q, &sm.qdo_full, s * 64, i * kTile, bh);
         tma_load_3d(sm.dout + s * kTile * 64, &tm_do, &sm.qdo_full, s * 64, i * kTile, bh);
       }
-      for (int pass = 0; pass < 2 && ok; ++pass) {
+      {
         for (int t = 0; t < n && ok; ++t) {
           const int j = sm.tiles[t];
           {
@@ -272,7 +277,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t kcm = 0, vcm = 0;        // K / V tiles consumed
       uint32_t ks_of0 = 0, ks_of1 = 0;  // K slot of the tile each buffer's step belongs to
       // S = Q K_h^T and dP = dO V_h^T of step `step` (half h of the current tile)
-      auto issue_sdp = [&](bool release_k) -> bool {
+      auto issue_sdp = [&]() -> bool {
         const uint32_t h = step & 1, use = step >> 1;
         const uint32_t ks = kcm % NSK, vs = vcm % NSV;
         if (h == 0) {
@@ -296,7 +301,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         else ks_of1 = ks;
         if (h == 1) {
           mma_commit(&sm.v_empty[vs]);
-          if (release_k) mma_commit(&sm.k_empty[ks]);
           ++kcm;
           ++vcm;
         }
@@ -322,11 +326,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ++dstep;
         return true;
       };
-      // pass A: delta
-      for (int u = 0; u < 2 * n && ok; ++u) ok = issue_sdp(true);
-      // pass B: dQ, dQ steps trail the S/dP steps by one
+      // dQ steps trail the S/dP steps by one
       for (int u = 0; u <= 2 * n && ok; ++u) {
-        if (u < 2 * n) ok = issue_sdp(false);
+        if (u < 2 * n) ok = issue_sdp();
         if (ok && u > 0) ok = issue_dq();
       }
       if (ok) mma_commit(&sm.dq_full);
@@ -346,79 +348,81 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float tau_r = row_ok ? P.tau[static_cast<size_t>(bh) * P.N + row] : INFINITY;
     bool ok = true;
     uint32_t use = 0;   // uses of this warpgroup's S/dP buffer
-    float delta = 0.0f;
     uint8_t* ds_base = reinterpret_cast<uint8_t*>(sm.ds[wg]);
 
-    for (int pass = 0; pass < 2 && ok; ++pass) {
-      float gdp[4] = {0.f, 0.f, 0.f, 0.f}, gsm[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int t = 0; t < n; ++t) {
-        const int j = sm.tiles[t];
-        ok = mbar_wait(&sm.s_full[wg], use & 1, abort_flag, P.status);
-        // pass B, tile t >= 1: the dQ MMA of tile t - 1 must have read this dS buffer
-        if (ok && pass == 1 && use > static_cast<uint32_t>(n))
-          ok = mbar_wait(&sm.ds_empty[wg], (use - n - 1) & 1, abort_flag, P.status);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        ++use;
-        tc_fence_after();
-        const int col0 = j * kTile + wg * kHalf;
-        const bool msk = (P.causal && j == i) || (col0 + kHalf > P.N);
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t rs[32], rp[32];
-          tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
-          if (ch == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_empty[wg]);
-          }
-          float gg[32];
+    // delta of the row: warpgroup wg takes dimensions [wg D/2, (wg + 1) D/2)
+    {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      if (row_ok) {
+        const size_t off = (static_cast<size_t>(bh) * P.N + row) * D + wg * (D / 2);
+        const uint4* dsrc = reinterpret_cast<const uint4*>(P.dout16 + off);
+        const float4* vsrc = reinterpret_cast<const float4*>(P.vbar + off);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float tt = fmaf(__uint_as_float(rs[e]), P.c, -tau_r);
+        for (int u = 0; u < D / 16; ++u) {
+          const uint4 hv = dsrc[u];
+          const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float4 vb = vsrc[2 * u + h];
+            const float2 d0 = __half22float2(*reinterpret_cast<const __half2*>(&hw[2 * h]));
+            const float2 d1 = __half22float2(*reinterpret_cast<const __half2*>(&hw[2 * h + 1]));
+            acc[2 * h] = fmaf(d0.x, vb.x, fmaf(d0.y, vb.y, acc[2 * h]));
+            acc[2 * h + 1] = fmaf(d1.x, vb.z, fmaf(d1.y, vb.w, acc[2 * h + 1]));
+          }
+        }
+      }
+      sm.part_delta[wg][rl] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      bwd_epi_bar();
+    }
+    const float delta = sm.part_delta[0][rl] + sm.part_delta[1][rl];
+    if (row_ok && wg == 0) P.delta[static_cast<size_t>(bh) * P.N + row] = delta;
+
+    for (int t = 0; t < n; ++t) {
+      const int j = sm.tiles[t];
+      ok = mbar_wait(&sm.s_full[wg], use & 1, abort_flag, P.status);
+      // tile t >= 1: the dQ MMA of tile t - 1 must have read this dS buffer
+      if (ok && use > 0) ok = mbar_wait(&sm.ds_empty[wg], (use - 1) & 1, abort_flag, P.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++use;
+      tc_fence_after();
+      const int col0 = j * kTile + wg * kHalf;
+      const bool msk = (P.causal && j == i) || (col0 + kHalf > P.N);
+#pragma unroll 1
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t rs[32], rp[32];
+        tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
+        if (ch == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_empty[wg]);
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float g2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            float tt = fmaf(__uint_as_float(rs[2 * e + u]), P.c, -tau_r);
             if (msk) {
-              const int col = col0 + ch * 32 + e;
+              const int col = col0 + ch * 32 + 2 * e + u;
               if (!(col < P.N && (!P.causal || col <= row))) tt = -1.0f;
             }
-            gg[e] = ALPHA2 ? (tt > 0.f ? 1.f : 0.f) : fmaxf(tt, 0.f);
+            g2[u] = ALPHA2 ? (tt > 0.f ? 1.f : 0.f) : fmaxf(tt, 0.f);
           }
-          if (pass == 0) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              gdp[e & 3] = fmaf(gg[e], __uint_as_float(rp[e]), gdp[e & 3]);
-              gsm[e & 3] += gg[e];
-            }
-          } else {
-            uint32_t w[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float d0 = gg[2 * e] * (__uint_as_float(rp[2 * e]) - delta);
-              const float d1 = gg[2 * e + 1] * (__uint_as_float(rp[2 * e + 1]) - delta);
-              const __half2 h2 = __floats2half2_rn(d0, d1);
-              w[e] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd)
-              *reinterpret_cast<uint4*>(ds_base + sw128_chunk_offset(rl, ch * 4 + qd)) =
-                  make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
-          }
+          const float d0 = g2[0] * (__uint_as_float(rp[2 * e]) - delta);
+          const float d1 = g2[1] * (__uint_as_float(rp[2 * e + 1]) - delta);
+          const __half2 h2 = __floats2half2_rn(d0, d1);
+          w[e] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        if (pass == 1) {
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.ds_full[wg]);
-        }
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd)
+          *reinterpret_cast<uint4*>(ds_base + sw128_chunk_offset(rl, ch * 4 + qd)) =
+              make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
       }
-      if (pass == 0) {
-        // combine the two warpgroups' partial sums of the row: delta = sum g dP / sum g
-        sm.part_gdp[wg][rl] = (gdp[0] + gdp[1]) + (gdp[2] + gdp[3]);
-        sm.part_g[wg][rl] = (gsm[0] + gsm[1]) + (gsm[2] + gsm[3]);
-        bwd_epi_bar();
-        const float a = sm.part_gdp[0][rl] + sm.part_gdp[1][rl];
-        const float g = sm.part_g[0][rl] + sm.part_g[1][rl];
-        delta = g > 0.f ? a / g : 0.0f;
-        if (row_ok && wg == 0) P.delta[static_cast<size_t>(bh) * P.N + row] = delta;
-      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.ds_full[wg]);
     }
     // dQ epilogue: warpgroup wg stores columns [wg * D/2, (wg + 1) * D/2)
     if (ok && n > 0) {

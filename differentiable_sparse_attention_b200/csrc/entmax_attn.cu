@@ -27,7 +27,8 @@ struct WsLayout {
   size_t tilemask = 0;   // uint32 [BH][T][ceil(T/32)] 128-granularity mask
   size_t tilemaskT = 0;  // uint32 [BH][T][ceil(T/32)] its transpose
   size_t delta = 0;      // float [BH][N]
-  size_t half_copies = 0;  // fp16 copies of q, k, v, dout for the backward
+  size_t vbar = 0;       // float [BH][N][D] g-weighted means of v (forward -> backward)
+  size_t half_copies = 0;  // fp16 copies of q, k, v (made by the forward), dout
   size_t total = 0;
 };
 
@@ -48,6 +49,8 @@ WsLayout ws_layout(int B, int H, int N, int D, int causal) {
   off = align256(off + bh * t * words * sizeof(uint32_t));
   L.delta = off;
   off = align256(off + bh * static_cast<size_t>(N) * sizeof(float));
+  L.vbar = off;
+  off = align256(off + bh * static_cast<size_t>(N) * D * sizeof(float));
   L.half_copies = off;
   off = align256(off + 4 * bh * static_cast<size_t>(N) * D * sizeof(__half));
   L.total = off;
@@ -121,6 +124,15 @@ template <typename Kernel>
 bool set_smem(Kernel k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(bytes)) == cudaSuccess;
+}
+
+// dst = src in fp16 (exact for bf16 values within the fp16 range; others set
+// ENTMAX_ST_RANGE in *status).  D is a multiple of 8, so elems is too.
+void launch_to_fp16(const __nv_bfloat16* src, __half* dst, size_t elems, uint32_t* status,
+                    cudaStream_t st) {
+  const size_t n8 = elems / 8;
+  const int grid = static_cast<int>(std::min<size_t>((n8 + 255) / 256, 148 * 8));
+  to_fp16_kernel<<<grid, 256, 0, st>>>(src, dst, n8, status);
 }
 
 template <int D, int NS, bool A2>
@@ -279,8 +291,16 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
     prof_mark(EV_FWD1, st);
     return rc;
   }
+  // P.V and G.V run on an exact fp16 copy of v, which the backward reuses.
+  const size_t elems = static_cast<size_t>(BH) * N * D;
+  __half* v16 = reinterpret_cast<__half*>(ws + L.half_copies) + 2 * elems;
+  prof_mark(EV_FWD0, st);
+  launch_to_fp16(static_cast<const __nv_bfloat16*>(v), v16, elems,
+                 reinterpret_cast<uint32_t*>(ws + L.status), st);
+  if (cudaGetLastError() != cudaSuccess) return ENTMAX_E_CUDA;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) ||
+      !make_map(&mv, v16, BH, N, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return ENTMAX_E_CUDA;
 
   FwdParams p{};
@@ -304,9 +324,9 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
   p.inv_c = std::nextafter(1.0f / p.c, INFINITY) * (1.0f + 1e-6f);
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
+  p.vbar = reinterpret_cast<float*>(ws + L.vbar);
 
   const bool a2 = alpha == 2.0f;
-  prof_mark(EV_FWD0, st);
   if (D == 64) {
     rc = a2 ? launch_fwd<64, 3, true>(mq, mk, mv, p, st) : launch_fwd<64, 3, false>(mq, mk, mv, p, st);
   } else {
@@ -363,6 +383,7 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, 
   p.tau = tau;
   p.mask = mask;
   p.tau_trace = nullptr;
+  p.vbar = nullptr;   // no room for the g-weighted means: P.V in bf16 on v itself
   p.tmax = reinterpret_cast<__half*>(ws + L.tmax);
   p.inv_c = std::nextafter(1.0f / p.c, INFINITY) * (1.0f + 1e-6f);
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
@@ -419,10 +440,9 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
   const void* srcs[4] = {q, k, v, dout};
   for (int a = 0; a < 4; ++a) {
     h16[a] = reinterpret_cast<__half*>(ws + L.half_copies) + a * elems;
-    const size_t n8 = elems / 8;  // D is a multiple of 8
-    const int grid = static_cast<int>(std::min<size_t>((n8 + 255) / 256, 148 * 8));
-    to_fp16_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(srcs[a]), h16[a], n8,
-                                         status_word);
+    // v's copy was made by the forward
+    if (a != 2)
+      launch_to_fp16(static_cast<const __nv_bfloat16*>(srcs[a]), h16[a], elems, status_word, st);
   }
   if (cudaGetLastError() != cudaSuccess) return ENTMAX_E_CUDA;
   prof_mark(EV_BWD_CONV, st);
@@ -458,6 +478,8 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
   p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(D));
   p.tau = tau;
   p.delta = reinterpret_cast<float*>(ws + L.delta);
+  p.vbar = reinterpret_cast<const float*>(ws + L.vbar);
+  p.dout16 = h16[3];
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);

@@ -51,6 +51,10 @@ struct FwdParams {
   float inv_c;               // 1 / c rounded up
   uint32_t* status;          // workspace word 0
   unsigned long long* counters;  // workspace, CNT_* work counters
+  // nullable, [BH][N][D]: g-weighted mean of v per row, sum_c g v_c / sum_c g
+  // with g = p^(2 - alpha).  Non-null: V is an fp16 copy and P, G are fp16;
+  // null: V is the bf16 input, P is bf16 and G is not formed.
+  float* vbar;
 };
 
 // tau_h: exact root of the reduced histogram problem.  cnt[b] counts the scores
@@ -181,15 +185,14 @@ struct FwdSmem {
   __nv_bfloat16 q[kTile * D];       // D/64 swizzled slabs
   __nv_bfloat16 k[NS][kTile * D];
   __nv_bfloat16 v[NS][kTile * D];
-  // P tiles, K-major (K = keys), 2 slabs each (slab h written by warpgroup h);
-  // double-buffered when D = 64 leaves room
+  // candidate storage beyond the V ring (P and G of the P.V pass live in TMEM)
   static constexpr int kNSP = D == 64 ? 2 : 1;
   __nv_bfloat16 p[kNSP][kTile * kTile];
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS];
   uint64_t v_full[NS], v_empty[NS];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[kNSP], p_empty[kNSP], o_full, drain;
+  uint64_t p_full[2], p_empty[2], o_full, drain;
   uint32_t tmem_base;
   int abort_flag;
   int ctl_kind, ctl_n, ctl_iter;
@@ -202,6 +205,7 @@ struct FwdSmem {
   FwdXrow x1[kTile];          // 1 -> 0: histogram / candidate state
   double xf[3][kTile];        // 1 -> 0: refinement partial sums
   float xtmin[kTile], xtneg[kTile], xsum[kTile];
+  float xg[2][kTile];         // both: partial sums of g per warpgroup
   double xlo[kTile];          // 0 -> 1: bracket lower bound
   float xtau[kTile];          // 0 -> 1: current threshold
   int xflag[kTile];           // 0 -> 1: list rebuilt by COLLECT
@@ -223,6 +227,8 @@ template <int D, int NS>
 constexpr size_t fwd_smem_bytes() {
   return sizeof(FwdSmem<D, NS>) + 1024;  // + slack for 1024-byte alignment
 }
+static_assert(fwd_smem_bytes<64, 3>() <= 232448 && fwd_smem_bytes<128, 2>() <= 232448,
+              "forward shared memory above the 227 KB per block");
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);
@@ -249,9 +255,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   constexpr int kSlabs = D / 64;
   constexpr uint32_t kTileBytes = kTile * D * 2;
   constexpr uint32_t kIdescS = make_idesc(kTile, kTile, 1, 1, 0, 0);  // Q (K-major) x K (K-major)
-  constexpr uint32_t kIdescPV = make_idesc(kTile, D, 1, 1, 0, 1);     // P (K-major) x V (MN-major)
-  constexpr uint32_t kColO = 256;                                     // TMEM: S0, S1, O
-  constexpr uint32_t kNSP = Smem::kNSP;
+  // P / G (TMEM) x V (SMEM, MN-major): fp16 with the g-weighted means, else bf16
+  const uint32_t idesc_pv = P.vbar != nullptr ? make_idesc(kTile, D, 0, 0, 0, 1)
+                                              : make_idesc(kTile, D, 1, 1, 0, 1);
+  const bool gv = P.vbar != nullptr;
+  constexpr uint32_t kColO = 256;      // TMEM: S0, S1 (P / G of the P.V pass), O, G.V
+  constexpr uint32_t kColG = 256 + D;
   constexpr int kCap = fwd_cand_cap<D, NS>();
   constexpr int kCapH = kCap / 2;
   static_assert(offsetof(Smem, p) == offsetof(Smem, v) + NS * kTile * D * 2,
@@ -276,7 +285,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.s_empty[s], 8);
     }
-    for (int s = 0; s < static_cast<int>(kNSP); ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.p_full[s], 8);
       mbar_init(&sm.p_empty[s], 1);
     }
@@ -348,6 +357,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   int iter = 0;
   bool row_done = false;                   // threshold certified exact
   float rowsum = 0.0f;
+  float gsum = 0.0f;                       // sum of g = p^(2 - alpha) over this half
 
   auto trace_store = [&](int it, float val) {
     if (P.tau_trace != nullptr && row_ok && wg == 0 && it <= P.max_iter)
@@ -444,21 +454,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ++sc;
           return true;
         };
-        auto issue_pv = [&]() -> bool {
-          const uint32_t pb = pc % kNSP;
-          if (!mbar_wait(&sm.p_full[pb], (pc / kNSP) & 1, abort_flag, P.status)) return false;
+        // O += P V and (with the g-weighted means) G.V += G V for P.V tile pc.
+        // P and G sit in the S buffer of their tile: 32-key chunk c occupies
+        // columns 32 c .. 32 c + 31, P packed in the first 16, G in the last 16.
+        auto issue_pv = [&](uint32_t sc0) -> bool {
+          const uint32_t pb = pc & 1;
+          if (!mbar_wait(&sm.p_full[pb], (pc >> 1) & 1, abort_flag, P.status)) return false;
           const uint32_t slot = vc % NS;
           if (!mbar_wait(&sm.v_full[slot], (vc / NS) & 1, abort_flag, P.status)) return false;
           tc_fence_after();
-          const uint32_t p_addr = smem_u32(sm.p[pb]);
+          const uint32_t t_p = tmem + ((sc0 + pc) & 1) * kTile;
           const uint32_t v_addr = smem_u32(sm.v[slot]);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint32_t a_off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-            const uint32_t b_off = kk * 16 * 128;  // 16 keys of 128-byte rows
-            mma_f16_ss(tmem + kColO, smem_desc_sw128(p_addr + a_off, 16, 1024),
-                       smem_desc_sw128(v_addr + b_off, kSlabBytes, 1024), kIdescPV,
-                       (pc > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t a_col = (kk >> 1) * 32 + (kk & 1) * 8;
+            const uint64_t vd = smem_desc_sw128(v_addr + kk * 16 * 128, kSlabBytes, 1024);
+            const uint32_t acc = (pc > 0 || kk > 0) ? 1u : 0u;
+            mma_f16_ts(tmem + kColO, t_p + a_col, vd, idesc_pv, acc);
+            if (gv) mma_f16_ts(tmem + kColG, t_p + a_col + 16, vd, idesc_pv, acc);
           }
           mma_commit(&sm.v_empty[slot]);
           mma_commit(&sm.p_empty[pb]);
@@ -470,9 +483,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (kind != PASS_PV) {
             for (int t = 0; t < n && ok; ++t) ok = issue_s();
           } else {
+            const uint32_t sc0 = sc;
             for (int t = 0; t <= n && ok; ++t) {
-              if (t < n) ok = issue_s();
-              if (ok && t > 0) ok = issue_pv();
+              // S(t) reuses the TMEM buffer of P.V tile t - 2: wait for its MMAs
+              if (t < n && t >= 2)
+                ok = mbar_wait(&sm.p_empty[t & 1], ((t - 2) >> 1) & 1, abort_flag, P.status);
+              if (ok && t < n) ok = issue_s();
+              if (ok && t > 0) ok = issue_pv(sc0);
             }
             if (ok) mma_commit(&sm.o_full);
           }
@@ -485,7 +502,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       double F0 = 0.0, F1 = 0.0, F2 = 0.0;  // refinement sums at tau_c (this half)
       float Tmin = INFINITY;                // smallest positive s - tau_c
       float Tneg = -INFINITY;               // largest non-positive s - tau_c
-      if (kind == PASS_PV) rowsum = 0.0f;
+      if (kind == PASS_PV) {
+        rowsum = 0.0f;
+        gsum = 0.0f;
+      }
       for (int t = 0; t < n; ++t) {
         const int j = sm.tiles[t];
         const uint32_t cur = sc++;
@@ -684,51 +704,55 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           Tmin = fminf(Tmin, fminf(fminf(tmin[0], tmin[1]), fminf(tmin[2], tmin[3])));
           Tneg = fmaxf(Tneg, fmaxf(fmaxf(tneg[0], tneg[1]), fmaxf(tneg[2], tneg[3])));
         } else {  // PASS_PV
-          const uint32_t cur_p = pc++;
-          const uint32_t pb = cur_p % kNSP, puse = cur_p / kNSP;
-          if (puse > 0) {
-            ok = mbar_wait(&sm.p_empty[pb], (puse - 1) & 1, abort_flag, P.status);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-          }
-          float part = 0.f;
-          uint8_t* p_base = reinterpret_cast<uint8_t*>(sm.p[pb]);
+          // P (and G) replace the scores in this S buffer; the MMA warp issues
+          // S(t + 2) into it only after the P.V MMAs of this tile completed.
+          const uint32_t pb = pc & 1;
+          ++pc;
+          float part = 0.f, gpart = 0.f;
 #pragma unroll 1
           for (int ch = 0; ch < 2; ++ch) {
             uint32_t r[32];
             tmem_ld32(t_s + ch * 32, r);
-            if (ch == 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
-            }
             float v[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (msk) apply_mask(v, j, ch);
-            uint32_t w[16];
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t w[16], wgt[16];
+            float ps[4] = {0.f, 0.f, 0.f, 0.f}, gs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const float t0 = fmaxf(fmaf(v[2 * e], P.c, -tau_c), 0.0f);
               const float t1 = fmaxf(fmaf(v[2 * e + 1], P.c, -tau_c), 0.0f);
               const float p0 = ALPHA2 ? t0 : t0 * t0;
               const float p1 = ALPHA2 ? t1 : t1 * t1;
+              // g = p^(2 - alpha): the support indicator at alpha = 2, t at 1.5
+              const float g0 = ALPHA2 ? (t0 > 0.0f ? 1.0f : 0.0f) : t0;
+              const float g1 = ALPHA2 ? (t1 > 0.0f ? 1.0f : 0.0f) : t1;
               ps[e & 3] += p0 + p1;
-              const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-              w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+              gs[e & 3] += g0 + g1;
+              if (gv) {
+                const __half2 h2 = __floats2half2_rn(p0, p1);
+                const __half2 g2 = __floats2half2_rn(g0, g1);
+                w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                wgt[e] = *reinterpret_cast<const uint32_t*>(&g2);
+              } else {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+              }
             }
             part += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-            // keys hc0 + 32 ch + 8 qd .. : slab wg of the K-major P tile
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-              *reinterpret_cast<uint4*>(p_base + sw128_chunk_offset(rl, wg * 8 + ch * 4 + qd)) =
-                  make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
-            }
+            gpart += (gs[0] + gs[1]) + (gs[2] + gs[3]);
+            tmem_st16(t_s + ch * 32, w);
+            if (gv) tmem_st16(t_s + ch * 32 + 16, wgt);
           }
-          fence_proxy_async_smem();
+          tmem_wait_st();
+          tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.p_full[pb]);
+          if (lane == 0) {
+            mbar_arrive(&sm.p_full[pb]);
+            mbar_arrive(&sm.s_empty[sb]);
+          }
+          gsum += gpart;
           rowsum += part;
           const uint32_t bits = __ballot_sync(0xffffffffu, row_ok && part > 0.f);
           if (lane == 0 && bits != 0u) {
@@ -973,6 +997,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ok = __all_sync(0xffffffffu, ok);
         }
         tc_fence_after();
+        if (wg == 1) sm.xsum[rl] = rowsum;
+        sm.xg[wg][rl] = gsum;
+        fwd_epi_bar();
+        const float gtot = sm.xg[0][rl] + sm.xg[1][rl];
         __nv_bfloat16* orow = P.out + (static_cast<size_t>(bh) * P.N + row) * D;
         // warpgroup wg stores O columns [wg D/2, (wg + 1) D/2)
 #pragma unroll 1
@@ -998,9 +1026,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               dst[qd] = make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
           }
         }
-        if (wg == 1) sm.xsum[rl] = rowsum;
+        if (gv) {
+          // g-weighted means of v: G.V / sum g, columns [wg D/2, (wg + 1) D/2)
+          const float inv_g = gtot > 0.0f ? 1.0f / gtot : 0.0f;
+          float* vrow = P.vbar + (static_cast<size_t>(bh) * P.N + row) * D;
+#pragma unroll 1
+          for (int ch = wg * (D / 64); ch < (wg + 1) * (D / 64); ++ch) {
+            uint32_t r[32];
+            if (ok && n > 0) {
+              tmem_ld32(t_lane + kColG + ch * 32, r);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) r[e] = 0u;
+            }
+            if (row_ok) {
+              float4* dst = reinterpret_cast<float4*>(vrow + ch * 32);
+#pragma unroll
+              for (int qd = 0; qd < 8; ++qd)
+                dst[qd] = make_float4(__uint_as_float(r[4 * qd]) * inv_g,
+                                      __uint_as_float(r[4 * qd + 1]) * inv_g,
+                                      __uint_as_float(r[4 * qd + 2]) * inv_g,
+                                      __uint_as_float(r[4 * qd + 3]) * inv_g);
+            }
+          }
+        }
         tc_fence_before();
-        fwd_epi_bar();
         if (wg == 0 && row_ok) {
           rowsum += sm.xsum[rl];
           P.tau[static_cast<size_t>(bh) * P.N + row] = tau_c;

@@ -85,11 +85,12 @@ int entmax_attn_mask_words(int N, int block);
 
 /*
  * Bytes of device workspace that entmax_attn_fwd and entmax_attn_bwd need for
- * this problem (the same buffer serves both).  It holds the status word and
- * work counters, the per-(row, key tile) score maxima of the histogram pass
- * (fp16, rounded up), the tile-granularity mask and its transpose, the
- * per-row delta of the backward and the backward's fp16 copies of q, k, v and
- * dout.
+ * this problem (the same buffer serves both, and carries data from the bf16
+ * forward to its backward).  It holds the status word and work counters, the
+ * per-(row, key tile) score maxima of the histogram pass (fp16, rounded up),
+ * the tile-granularity mask and its transpose, the per-row delta of the
+ * backward, the forward's per-row g-weighted means of v (float32, B*H*N*D)
+ * and fp16 copies of q, k, v and dout (v's made by the forward).
  * Returns 0 for unsupported arguments.
  */
 size_t entmax_attn_workspace_size(int B, int H, int N, int D, int block, int causal);
@@ -118,7 +119,13 @@ size_t entmax_attn_workspace_size(int B, int H, int N, int D, int block, int cau
  *                     entry 0 is the histogram bound tau_h, entry i the
  *                     threshold after refinement step i.
  *   workspace    in/out  device buffer of >= entmax_attn_workspace_size() bytes,
- *                     256-byte aligned; its status word is cleared here.
+ *                     256-byte aligned; its status word is cleared here.  For
+ *                     bf16 the forward also leaves there what its backward
+ *                     reads: an exact fp16 copy of v (the P.V products run on
+ *                     it; a v entry beyond the fp16 range raises
+ *                     ENTMAX_ST_RANGE) and, per row, the g-weighted mean of v,
+ *                     vbar_r = sum_c g_rc v_c / sum_c g_rc with g = p^(2-alpha),
+ *                     formed by one more MMA next to P.V.
  */
 int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int D,
                     int dtype, float alpha, int causal, int block, int max_iter, void* out,
@@ -168,7 +175,12 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, 
  *   alpha, causal, block   as given to entmax_attn_fwd.
  *   dq, dk, dv     out [B][H][N][D], dtype (fully overwritten).
  *   workspace      in/out  the same size rule as for the forward; status bits
- *                  are OR-ed into the existing status word.
+ *                  are OR-ed into the existing status word.  bf16: the
+ *                  workspace the forward of these same inputs wrote, unchanged
+ *                  since (delta_r = dO_r . vbar_r uses its g-weighted means of
+ *                  v, the MMAs its fp16 copy of v); anything else gives
+ *                  undefined gradients.  fp32 computes delta in a pass of its
+ *                  own and needs no forward data.
  * The backward's MMAs run on exact fp16 copies of the bf16 inputs, so that
  * the operands rounded on chip (P and dS) keep 11 significant bits; an input
  * of magnitude above 65504 (outside fp16) raises ENTMAX_ST_RANGE.

@@ -43,7 +43,9 @@ def test_backward_deterministic(cuda_device):
     w = Workload("det", B=1, H=4, N=1024, D=128, alpha=1.5, temperature=2.0, seed=5)
     x = make_inputs(w, device=cuda_device)
     f = entmax_attn_fwd(x["q"], x["k"], x["v"], 1.5, True, 128)
-    a = entmax_attn_bwd(x["q"], x["k"], x["v"], x["dout"], f.tau, f.mask, 1.5, True, 128)
-    b = entmax_attn_bwd(x["q"], x["k"], x["v"], x["dout"], f.tau, f.mask, 1.5, True, 128)
+    a = entmax_attn_bwd(x["q"], x["k"], x["v"], x["dout"], f.tau, f.mask, 1.5, True, 128,
+                        workspace=f.workspace)
+    b = entmax_attn_bwd(x["q"], x["k"], x["v"], x["dout"], f.tau, f.mask, 1.5, True, 128,
+                        workspace=f.workspace)
     for ga, gb in zip(a, b):
         assert torch.equal(ga, gb)

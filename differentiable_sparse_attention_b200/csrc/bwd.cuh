@@ -165,7 +165,6 @@ struct BwdRowSmem {
   __half dout[kTile * D];
   __half k[NSK][kTile * D];
   __half v[NSV][kTile * D];
-  __half ds[2][kTile * kHalf];       // dS half tiles [128 rows][64 keys], K-major
   float part_delta[2][kTile];        // half-dot products per warpgroup
   uint64_t qdo_full;
   uint64_t k_full[NSK], k_empty[NSK];
@@ -194,8 +193,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr int kSlabs = D / 64;
   constexpr uint32_t kTileBytes = kTile * D * 2;
   constexpr uint32_t kIdescS = make_idesc(kTile, kHalf, 0, 0, 0, 0);  // [128 x D] x [64 x D]^T
-  constexpr uint32_t kIdescDQ = make_idesc(kTile, D, 0, 0, 0, 1);     // dS half x K half (MN-major)
-  constexpr uint32_t kColDQ = 256;  // TMEM: buffer b holds S at 128 b, dP at 128 b + 64
+  constexpr uint32_t kIdescDQ = make_idesc(kTile, D, 0, 0, 0, 1);     // dS (TMEM) x K half (MN-major)
+  // TMEM: buffer b holds S at 128 b, dP at 128 b + 64; the epilogue overwrites
+  // S with dS (fp16, 32-key chunk c packed into columns 128 b + 32 c .. + 15)
+  constexpr uint32_t kColDQ = 256;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -284,7 +285,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!mbar_wait(&sm.k_full[ks], (kcm / NSK) & 1, abort_flag, P.status)) return false;
           if (!mbar_wait(&sm.v_full[vs], (vcm / NSV) & 1, abort_flag, P.status)) return false;
         }
+        // buffer h is free once its epilogue is done and the dQ MMA read its dS
         if (use > 0 && !mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
+        if (use > 0 && !mbar_wait(&sm.ds_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(sm.k[ks]) + h * (kHalf * 128);
         const uint32_t v_addr = smem_u32(sm.v[vs]) + h * (kHalf * 128);
@@ -313,11 +316,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!mbar_wait(&sm.ds_full[h], use & 1, abort_flag, P.status)) return false;
         tc_fence_after();
         const uint32_t ks = h == 0 ? ks_of0 : ks_of1;
-        const uint32_t ds_addr = smem_u32(sm.ds[h]);
         const uint32_t k_addr = smem_u32(sm.k[ks]) + h * (kHalf * 128);
 #pragma unroll
         for (int kk = 0; kk < kHalf / 16; ++kk) {
-          mma_f16_ss(tmem + kColDQ, smem_desc_sw128(ds_addr + kk * 32, 16, 1024),
+          const uint32_t a_col = 128 * h + (kk >> 1) * 32 + (kk & 1) * 8;
+          mma_f16_ts(tmem + kColDQ, tmem + a_col,
                      smem_desc_sw128(k_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescDQ,
                      (dstep > 0 || kk > 0) ? 1u : 0u);
         }
@@ -348,7 +351,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float tau_r = row_ok ? P.tau[static_cast<size_t>(bh) * P.N + row] : INFINITY;
     bool ok = true;
     uint32_t use = 0;   // uses of this warpgroup's S/dP buffer
-    uint8_t* ds_base = reinterpret_cast<uint8_t*>(sm.ds[wg]);
 
     // delta of the row: warpgroup wg takes dimensions [wg D/2, (wg + 1) D/2)
     {
@@ -380,8 +382,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int t = 0; t < n; ++t) {
       const int j = sm.tiles[t];
       ok = mbar_wait(&sm.s_full[wg], use & 1, abort_flag, P.status);
-      // tile t >= 1: the dQ MMA of tile t - 1 must have read this dS buffer
-      if (ok && use > 0) ok = mbar_wait(&sm.ds_empty[wg], (use - 1) & 1, abort_flag, P.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ++use;
@@ -392,11 +392,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int ch = 0; ch < 2; ++ch) {
         uint32_t rs[32], rp[32];
         tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
-        if (ch == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_empty[wg]);
-        }
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -415,14 +410,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const __half2 h2 = __floats2half2_rn(d0, d1);
           w[e] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-#pragma unroll
-        for (int qd = 0; qd < 4; ++qd)
-          *reinterpret_cast<uint4*>(ds_base + sw128_chunk_offset(rl, ch * 4 + qd)) =
-              make_uint4(w[4 * qd], w[4 * qd + 1], w[4 * qd + 2], w[4 * qd + 3]);
+        tmem_st16(t_s + ch * 32, w);   // dS over the S chunk just read
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.ds_full[wg]);
+      if (lane == 0) {
+        mbar_arrive(&sm.ds_full[wg]);
+        mbar_arrive(&sm.s_empty[wg]);
+      }
     }
     // dQ epilogue: warpgroup wg stores columns [wg * D/2, (wg + 1) * D/2)
     if (ok && n > 0) {
@@ -485,8 +481,6 @@ struct BwdColSmem {
   __half v[kTile * D];
   __half q[NS][kTile * D];
   __half dout[NS][kTile * D];
-  __half pt[2][kTile * kHalf];    // P^T half tiles  [128 keys][64 rows], K-major (K = rows)
-  __half dst[2][kTile * kHalf];   // dS^T half tiles [128 keys][64 rows]
   float tau[NS][kTile];
   float delta[NS][kTile];
   uint64_t kv_full;
@@ -515,7 +509,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr uint32_t kTileBytes = kTile * D * 2;
   constexpr uint32_t kIdescS = make_idesc(kTile, kHalf, 0, 0, 0, 0);   // K Q_h^T, V dO_h^T
   constexpr uint32_t kIdescAcc = make_idesc(kTile, D, 0, 0, 0, 1);    // P^T_h dO_h, dS^T_h Q_h
-  constexpr uint32_t kColDV = 256, kColDK = 256 + D;  // buffer b: S^T at 128 b, dP^T at 128 b + 64
+  // TMEM buffer b: S^T at 128 b, dP^T at 128 b + 64; the epilogue overwrites
+  // them with P^T and dS^T (fp16, 32-row chunk c packed into columns 32 c .. + 15)
+  constexpr uint32_t kColDV = 256, kColDK = 256 + D;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -607,7 +603,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto issue_s = [&](uint32_t u) -> bool {
         const uint32_t t = u >> 1, h = u & 1, slot = t % NS, use = u >> 1;
         if (h == 0 && !mbar_wait(&sm.q_full[slot], (t / NS) & 1, abort_flag, P.status)) return false;
+        // buffer h is free once its epilogue is done and dV / dK read P^T / dS^T
         if (use > 0 && !mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
+        if (use > 0 && !mbar_wait(&sm.pt_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm.q[slot]) + h * (kHalf * 128);
         const uint32_t do_addr = smem_u32(sm.dout[slot]) + h * (kHalf * 128);
@@ -628,13 +626,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm.q[slot]) + h * (kHalf * 128);
         const uint32_t do_addr = smem_u32(sm.dout[slot]) + h * (kHalf * 128);
-        const uint32_t pt_addr = smem_u32(sm.pt[h]), ds_addr = smem_u32(sm.dst[h]);
 #pragma unroll
         for (int kk = 0; kk < kHalf / 16; ++kk) {
           const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
-          mma_f16_ss(tmem + kColDV, smem_desc_sw128(pt_addr + kk * 32, 16, 1024),
+          const uint32_t a_col = 128 * h + (kk >> 1) * 32 + (kk & 1) * 8;
+          mma_f16_ts(tmem + kColDV, tmem + a_col,
                      smem_desc_sw128(do_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescAcc, acc);
-          mma_f16_ss(tmem + kColDK, smem_desc_sw128(ds_addr + kk * 32, 16, 1024),
+          mma_f16_ts(tmem + kColDK, tmem + a_col + kHalf,
                      smem_desc_sw128(q_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescAcc, acc);
         }
         mma_commit(&sm.pt_empty[h]);
@@ -663,14 +661,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const uint32_t t_s = t_lane + 128 * wg, t_dp = t_s + kHalf;
     bool ok = true;
-    uint8_t* pt_base = reinterpret_cast<uint8_t*>(sm.pt[wg]);
-    uint8_t* ds_base = reinterpret_cast<uint8_t*>(sm.dst[wg]);
     for (int t = 0; t < n; ++t) {
       const int it = sm.tiles[t];
       const uint32_t slot = t % NS;
       ok = mbar_wait(&sm.s_full[wg], t & 1, abort_flag, P.status) &&
            mbar_wait(&sm.q_full[slot], (t / NS) & 1, abort_flag, P.status);
-      if (ok && t > 0) ok = mbar_wait(&sm.pt_empty[wg], (t - 1) & 1, abort_flag, P.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -680,11 +675,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int ch = 0; ch < 2; ++ch) {
         uint32_t rs[32], rp[32];
         tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
-        if (ch == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_empty[wg]);
-        }
         uint32_t wp[16], wd[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -716,18 +706,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           wd[e / 2] = *reinterpret_cast<uint32_t*>(&b0);
           wd[e / 2 + 1] = *reinterpret_cast<uint32_t*>(&b1);
         }
-#pragma unroll
-        for (int qd = 0; qd < 4; ++qd) {
-          const uint32_t off = sw128_chunk_offset(kl, ch * 4 + qd);
-          *reinterpret_cast<uint4*>(pt_base + off) =
-              make_uint4(wp[4 * qd], wp[4 * qd + 1], wp[4 * qd + 2], wp[4 * qd + 3]);
-          *reinterpret_cast<uint4*>(ds_base + off) =
-              make_uint4(wd[4 * qd], wd[4 * qd + 1], wd[4 * qd + 2], wd[4 * qd + 3]);
-        }
+        tmem_st16(t_s + ch * 32, wp);    // P^T over the S^T chunk just read
+        tmem_st16(t_dp + ch * 32, wd);   // dS^T over the dP^T chunk
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.pt_full[wg]);
+      if (lane == 0) {
+        mbar_arrive(&sm.pt_full[wg]);
+        mbar_arrive(&sm.s_empty[wg]);
+      }
     }
     if (ok && n > 0) {
       ok = mbar_wait(&sm.acc_full, 0, abort_flag, P.status);

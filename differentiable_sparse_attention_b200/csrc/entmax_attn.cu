@@ -499,12 +499,12 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
     rc = a2 ? launch_bwd_col<64, 3, true>(mq, mk, mv, mdo, pcol, st)
             : launch_bwd_col<64, 3, false>(mq, mk, mv, mdo, pcol, st);
   } else {
-    rc = a2 ? launch_bwd_row<128, 2, 1, true>(mq, mk, mv, mdo, prow, st)
-            : launch_bwd_row<128, 2, 1, false>(mq, mk, mv, mdo, prow, st);
+    rc = a2 ? launch_bwd_row<128, 2, 2, true>(mq, mk, mv, mdo, prow, st)
+            : launch_bwd_row<128, 2, 2, false>(mq, mk, mv, mdo, prow, st);
     if (rc != ENTMAX_OK) return rc;
     prof_mark(EV_BWD_ROW, st);
-    rc = a2 ? launch_bwd_col<128, 1, true>(mq, mk, mv, mdo, pcol, st)
-            : launch_bwd_col<128, 1, false>(mq, mk, mv, mdo, pcol, st);
+    rc = a2 ? launch_bwd_col<128, 2, true>(mq, mk, mv, mdo, pcol, st)
+            : launch_bwd_col<128, 2, false>(mq, mk, mv, mdo, pcol, st);
   }
   prof_mark(EV_BWD_COL, st);
   return rc;

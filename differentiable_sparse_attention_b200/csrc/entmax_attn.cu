@@ -322,6 +322,7 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
   p.tau_trace = tau_trace;
   p.tmax = reinterpret_cast<__half*>(ws + L.tmax);
   p.inv_c = std::nextafter(1.0f / p.c, INFINITY) * (1.0f + 1e-6f);
+  p.inv_c_dn = std::nextafter(1.0f / p.c, 0.0f) * (1.0f - 1e-6f);
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
   p.vbar = reinterpret_cast<float*>(ws + L.vbar);
@@ -386,6 +387,7 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, 
   p.vbar = nullptr;   // no room for the g-weighted means: P.V in bf16 on v itself
   p.tmax = reinterpret_cast<__half*>(ws + L.tmax);
   p.inv_c = std::nextafter(1.0f / p.c, INFINITY) * (1.0f + 1e-6f);
+  p.inv_c_dn = std::nextafter(1.0f / p.c, 0.0f) * (1.0f - 1e-6f);
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
 

@@ -49,6 +49,7 @@ struct FwdParams {
   float* tau_trace;          // nullable, [max_iter + 1][BH][N]
   __half* tmax;              // workspace: per-(row, key tile) maxima of s, rounded up
   float inv_c;               // 1 / c rounded up
+  float inv_c_dn;            // 1 / c rounded down
   uint32_t* status;          // workspace word 0
   unsigned long long* counters;  // workspace, CNT_* work counters
   // nullable, [BH][N][D]: g-weighted mean of v per row, sum_c g v_c / sum_c g
@@ -104,6 +105,33 @@ __device__ __forceinline__ R hist_threshold(const uint32_t (&cnt)[kNB + 1], int 
     rel = (S1s - sqrt(disc > R(0) ? disc : R(0))) / Cs;
   }
   return static_cast<R>(gtop - kNB) / kNB + rel;
+}
+
+// A lower bound of tau_h in s-units, cheaper than the exact root: for every b,
+// the C scores of bins b..kNB (first moment A = sum c_b' b') satisfy
+// sum c [x - tau]_+^k >= C (mean - tau)^k for tau <= x_b (each term is at least
+// (x - tau)^k there; Cauchy-Schwarz for k = 2, equality for k = 1), so the
+// reduced function is >= 1 at min(x_b, mean - C^(-1/k)) and tau_h lies above
+// it.  The maximum over b is tau_h itself at alpha = 2 and within a fraction
+// of a bin of it at 1.5.  Relative margins of 2e-6 cover the fp32 rounding
+// (rsqrtf is within 2 ulp).
+template <bool ALPHA2>
+__device__ __forceinline__ float hist_lower_bound(const uint32_t (&cnt)[kNB + 1], int gtop) {
+  float best = -INFINITY;
+  uint32_t cc = 0u, aa = 0u;
+#pragma unroll
+  for (int b = kNB; b >= 0; --b) {
+    cc += cnt[b];
+    aa += cnt[b] * static_cast<uint32_t>(b);
+    const float rs = rsqrtf(static_cast<float>(cc));
+    const float ic = rs * rs;
+    const float inv_k = ALPHA2 ? ic : rs;          // C^(-1/k)
+    const float mean = static_cast<float>(aa) * (1.0f / kNB) * ic;
+    const float rb = fminf(static_cast<float>(b) * (1.0f / kNB), mean * 0.999998f - inv_k * 1.000002f);
+    best = cc > 0u ? fmaxf(best, rb) : best;
+  }
+  best += static_cast<float>(gtop - kNB) * (1.0f / kNB);
+  return best - 2e-6f * fmaxf(1.0f, fabsf(best));
 }
 
 // Safety margin below tau_h that absorbs the rounding of s and tau (2^-20 |tau|).
@@ -591,14 +619,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (ch == 0) cmx0 = cm;
             else cmx1 = cm;
           }
-          // Candidates of this tile half: every score above acc_raw, raised to the
-          // partial histogram's tau_h (scores seen so far by this warpgroup)
-          // whenever a chunk reaches the current bound.
+          // Candidates of this tile half: every score above acc_raw, raised to a
+          // lower bound of the partial histogram's tau_h (scores seen so far by
+          // this warpgroup, so <= tau*) whenever a chunk reaches the current bound.
           {
             acc_raw = fmaxf(acc_raw, __fsub_rd(m_raw, P.inv_c));
             if (row_ok && !cand_over && gtop_set && fmaxf(cmx0, cmx1) > acc_raw) {
-              const double th = hist_threshold<ALPHA2>(cnt, gtop);
-              acc_raw = fmaxf(acc_raw, __double2float_rd((th - hist_margin(th)) / P.c));
+              const float lb = hist_lower_bound<ALPHA2>(cnt, gtop);   // s-units
+              acc_raw = fmaxf(acc_raw, lb * (lb >= 0.0f ? P.inv_c_dn : P.inv_c));
             }
           }
 #pragma unroll 1

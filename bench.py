@@ -37,8 +37,50 @@ sys.path.insert(0, ROOT)
 
 from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
 
+# DRAM bytes (read + write) per launch from one ncu capture, keyed by workload
+# and kernel, valid only for the kernel sources they were taken on (hash of
+# the package's csrc/); any other source reports traffic as null.
+TRAFFIC = {
+    ("alpha15_4k", "fwd"): {"bytes": 68198656, "src": "14fef42f86235835",
+                            "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
+    ("alpha15_4k", "bwd_row"): {"bytes": 109259776, "src": "14fef42f86235835",
+                                "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
+    ("alpha15_4k", "bwd_col"): {"bytes": 75314176, "src": "14fef42f86235835",
+                                "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
+}
+
+
+def kernel_source_hash() -> str:
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "differentiable_sparse_attention_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The maximum of x over the ranks of the default process group (x itself
+    without one); the tensor lives on `device` (a CUDA device under NCCL)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(eff_flop_per_step_per_rank: float, steps: int, world: int,
+                     ms_total_max: float) -> float:
+    """Weak scaling: every rank runs the full workload, so the job processed
+    world x the per-rank work in the slowest rank's time."""
+    return eff_flop_per_step_per_rank * steps * world / (ms_total_max * 1e-3) / 1e12
 
 
 def load_peaks():
@@ -202,11 +244,7 @@ def run_ours(args, points, rank, world, device):
                     phases[n] += v
         torch.cuda.synchronize(device)
         dsa.profile(False)
-        ms_sum = sum(ms_steps)
-        if world > 1:
-            t = torch.tensor([ms_sum], device=device)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms_sum = float(t.item())
+        ms_sum = max_over_ranks(sum(ms_steps), device)
         ms_step = ms_sum / args.steps
         eff = effective_flops(w)
         total_eff += eff * args.steps * world
@@ -239,11 +277,7 @@ def run_ours(args, points, rank, world, device):
                 ev1.record()
                 ev1.synchronize()
                 e_ms.append(ev0.elapsed_time(ev1))
-            e_sum = sum(e_ms)
-            if world > 1:
-                t = torch.tensor([e_sum], device=device)
-                torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-                e_sum = float(t.item())
+            e_sum = max_over_ranks(sum(e_ms), device)
             e2e_ms += e_sum
             h2d += in_bytes
             d2h += out_bytes
@@ -267,6 +301,10 @@ def run_ours(args, points, rank, world, device):
     dom = max(phase_tot, key=phase_tot.get)
     dom_ms = phase_tot[dom] / n_steps_all
     roof = roofline_for(dom, dom_ms, points, results, peaks, peaks_kind, args.steps)
+    tr = TRAFFIC.get((args.workload, dom))
+    if tr is not None and not args.heads and tr["src"] == kernel_source_hash():
+        roof["traffic"] = tr["bytes"]
+        roof["traffic_from"] = tr["from"]
 
     line = {
         "metric": "fwd+bwd alpha-entmax attn ms/step & effective TFLOP/s vs block sparsity, 1 B200",

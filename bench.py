@@ -302,7 +302,8 @@ def run_ours(args, points, rank, world, device):
     dom_ms = phase_tot[dom] / n_steps_all
     roof = roofline_for(dom, dom_ms, points, results, peaks, peaks_kind, args.steps)
     tr = TRAFFIC.get((args.workload, dom))
-    if tr is not None and not args.heads and tr["src"] == kernel_source_hash():
+    if (tr is not None and not args.heads and not args.alpha
+            and tr["src"] == kernel_source_hash()):
         roof["traffic"] = tr["bytes"]
         roof["traffic_from"] = tr["from"]
 
@@ -448,10 +449,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (small cases for profiler captures)")
+    ap.add_argument("--alpha", type=float, default=0.0,
+                    help="override alpha (any value in [1.05, 3]; 1.5 and 2 have closed forms)")
     args = ap.parse_args()
     points = workload_points(args.workload)
     if args.heads:
         points = [p.with_(H=args.heads) for p in points]
+    if args.alpha:
+        points = [p.with_(alpha=args.alpha, name=f"{p.name}_as_alpha{args.alpha:g}") for p in points]
     args.workload_desc = (f"{args.workload}: " + ", ".join(
         f"B={p.B} H={p.H} N={p.N} D={p.D} alpha={p.alpha} t={p.temperature}"
         + (f" planted={p.planted_blocks}" if p.planted_blocks else "") for p in points)

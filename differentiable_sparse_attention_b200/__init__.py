@@ -126,11 +126,18 @@ def alloc_workspace(B, H, N, D, block=128, causal=True, device="cuda"):
     return torch.empty(workspace_size(B, H, N, D, block, causal), dtype=torch.uint8, device=device)
 
 
+def default_max_iter(alpha: float) -> int:
+    """Refinement cap: the closed forms (alpha 1.5 and 2) certify exactness within
+    one or two steps; the power path for other alpha stops on a tolerance."""
+    return 4 if float(alpha) in (1.5, 2.0) else 12
+
+
 def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = True, block: int = 128,
-                    max_iter: int = 4, *, out=None, tau=None, mask=None, workspace=None,
+                    max_iter=None, *, out=None, tau=None, mask=None, workspace=None,
                     trace: bool = False, stream=None) -> FwdResult:
     """alpha-entmax attention forward through ``entmax_attn_fwd``."""
     _check_qkv(q, k, v)
+    max_iter = default_max_iter(alpha) if max_iter is None else int(max_iter)
     B, H, N, D = q.shape
     dev = q.device
     out = torch.empty_like(q) if out is None else out
@@ -218,7 +225,7 @@ class EntmaxAttention(torch.autograd.Function):
     """autograd wrapper: O = entmax_attention(q, k, v); backward through the library."""
 
     @staticmethod
-    def forward(ctx, q, k, v, alpha=1.5, causal=True, block=128, max_iter=4):
+    def forward(ctx, q, k, v, alpha=1.5, causal=True, block=128, max_iter=None):
         r = entmax_attn_fwd(q, k, v, alpha, causal, block, max_iter)
         ctx.save_for_backward(q, k, v, r.tau, r.mask, r.workspace)
         ctx.cfg = (alpha, causal, block)
@@ -233,5 +240,5 @@ class EntmaxAttention(torch.autograd.Function):
         return dq, dk, dv, None, None, None, None
 
 
-def entmax_attention(q, k, v, alpha=1.5, causal=True, block=128, max_iter=4):
+def entmax_attention(q, k, v, alpha=1.5, causal=True, block=128, max_iter=None):
     return EntmaxAttention.apply(q, k, v, alpha, causal, block, max_iter)

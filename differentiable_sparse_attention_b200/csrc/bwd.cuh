@@ -105,6 +105,7 @@ struct BwdParams {
   int causal;
   float c;                   // (alpha - 1) / sqrt(D)
   float inv_sqrt_d;
+  float kpow;                // k = 1 / (alpha - 1), used by the generic-alpha kernels
   const float* tau;          // [BH][N]
   const uint32_t* tm;        // tile mask rows (row kernel) or transposed rows (column kernel)
   float* delta;              // workspace [BH][N]
@@ -181,13 +182,15 @@ constexpr size_t bwd_row_smem_bytes() {
   return sizeof(BwdRowSmem<D, NSK, NSV>) + 1024;
 }
 
-template <int D, int NSK, int NSV, bool ALPHA2>
+template <int D, int NSK, int NSV, int AM>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     entmax_bwd_row_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_do, const BwdParams P) {
   static_assert(NSK >= 2, "K(t - 1) stays for its dQ step while S(t) is issued");
+  constexpr bool ALPHA2 = AM == AM_2;
+  constexpr bool GEN = AM == AM_GEN;
   extern __shared__ uint8_t smem_raw[];
   auto& sm = *reinterpret_cast<BwdRowSmem<D, NSK, NSV>*>(align1024(smem_raw));
   constexpr int kSlabs = D / 64;
@@ -403,7 +406,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               const int col = col0 + ch * 32 + 2 * e + u;
               if (!(col < P.N && (!P.causal || col <= row))) tt = -1.0f;
             }
-            g2[u] = ALPHA2 ? (tt > 0.f ? 1.f : 0.f) : fmaxf(tt, 0.f);
+            if (GEN)   // g = t^(k - 1) <= 1 (alpha <= 2: k >= 1, t <= 1)
+              g2[u] = tt > 0.f ? __fdividef(pow_pos(tt, P.kpow), tt) : 0.f;
+            else
+              g2[u] = ALPHA2 ? (tt > 0.f ? 1.f : 0.f) : fmaxf(tt, 0.f);
           }
           const float d0 = g2[0] * (__uint_as_float(rp[2 * e]) - delta);
           const float d1 = g2[1] * (__uint_as_float(rp[2 * e + 1]) - delta);
@@ -497,12 +503,14 @@ constexpr size_t bwd_col_smem_bytes() {
   return sizeof(BwdColSmem<D, NS>) + 1024;
 }
 
-template <int D, int NS, bool ALPHA2>
+template <int D, int NS, int AM>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     entmax_bwd_col_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_do, const BwdParams P) {
+  constexpr bool ALPHA2 = AM == AM_2;
+  constexpr bool GEN = AM == AM_GEN;
   extern __shared__ uint8_t smem_raw[];
   auto& sm = *reinterpret_cast<BwdColSmem<D, NS>*>(align1024(smem_raw));
   constexpr int kSlabs = D / 64;
@@ -693,8 +701,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (!ok_e) tt = -1.0f;
             }
             const float tp = fmaxf(tt, 0.0f);
-            const float g = ALPHA2 ? (tt > 0.f ? 1.f : 0.f) : tp;
-            pp[u] = ALPHA2 ? tp : tp * tp;
+            float g;
+            if (GEN) {
+              pp[u] = pow_pos(tt, P.kpow);
+              g = tt > 0.f ? __fdividef(pp[u], tt) : 0.f;
+            } else {
+              g = ALPHA2 ? (tt > 0.f ? 1.f : 0.f) : tp;
+              pp[u] = ALPHA2 ? tp : tp * tp;
+            }
             dd[u] = g * (__uint_as_float(rp[e + u]) - dels[u]);
           }
           __half2 a0 = __floats2half2_rn(pp[0], pp[1]);

@@ -21,6 +21,16 @@ constexpr int kNB = 8;                       // histogram bins per unit of s
 constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23
 constexpr uint32_t kMagicBits = 0x4B400000u; // bit pattern of kMagic
 
+// alpha: the closed forms of 1.5 (p = t^2) and 2 (p = t), or any other alpha in
+// [1.05, 3] through powers t^k, k = 1 / (alpha - 1).
+enum AlphaMode : int { AM_15 = 0, AM_2 = 1, AM_GEN = 2 };
+
+// t^e for t > 0 (0 otherwise) from the base-2 logarithm and exponential of the
+// special-function unit: relative error about |e log2 t| 2^-22.
+__device__ __forceinline__ float pow_pos(float t, float e) {
+  return t > 0.0f ? exp2f(e * __log2f(t)) : 0.0f;
+}
+
 enum PassKind : int { PASS_HIST = 0, PASS_REFINE = 1, PASS_PV = 2, PASS_DONE = 3, PASS_COLLECT = 4 };
 
 // Work counters kept in the workspace right after the status word (uint64 each).

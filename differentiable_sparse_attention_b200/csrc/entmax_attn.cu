@@ -67,7 +67,9 @@ int check_common(int B, int H, int N, int D, int dtype, float alpha, int block) 
   if (dtype != ENTMAX_DTYPE_BF16 && dtype != ENTMAX_DTYPE_FP32) return ENTMAX_E_UNSUPPORTED;
   if (dtype == ENTMAX_DTYPE_FP32 && D != kF32D) return ENTMAX_E_UNSUPPORTED;
   if (block != 64 && block != 128) return ENTMAX_E_UNSUPPORTED;
-  if (!(alpha == 1.5f || alpha == 2.0f)) return ENTMAX_E_ALPHA;
+  // closed forms at 1.5 and 2, powers t^k for the rest of [1.05, 3]
+  if (!(alpha >= 1.05f && alpha <= 3.0f)) return ENTMAX_E_ALPHA;
+  if (dtype == ENTMAX_DTYPE_FP32 && !(alpha == 1.5f || alpha == 2.0f)) return ENTMAX_E_UNSUPPORTED;
   return ENTMAX_OK;
 }
 
@@ -135,10 +137,10 @@ void launch_to_fp16(const __nv_bfloat16* src, __half* dst, size_t elems, uint32_
   to_fp16_kernel<<<grid, 256, 0, st>>>(src, dst, n8, status);
 }
 
-template <int D, int NS, bool A2>
+template <int D, int NS, int AM>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const FwdParams& p, cudaStream_t st) {
-  auto kern = entmax_fwd_kernel<D, NS, A2>;
+  auto kern = entmax_fwd_kernel<D, NS, AM>;
   constexpr size_t smem = fwd_smem_bytes<D, NS>();
   static_assert(smem <= 232448, "forward kernel shared memory");
   static bool attr_ok = set_smem(kern, smem);
@@ -148,10 +150,10 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
 }
 
-template <int D, int NSK, int NSV, bool A2>
+template <int D, int NSK, int NSV, int AM>
 int launch_bwd_row(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                    const CUtensorMap& mdo, const BwdParams& p, cudaStream_t st) {
-  auto kern = entmax_bwd_row_kernel<D, NSK, NSV, A2>;
+  auto kern = entmax_bwd_row_kernel<D, NSK, NSV, AM>;
   constexpr size_t smem = bwd_row_smem_bytes<D, NSK, NSV>();
   static_assert(smem <= 232448, "bwd row kernel shared memory");
   static bool attr_ok = set_smem(kern, smem);
@@ -161,10 +163,10 @@ int launch_bwd_row(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
 }
 
-template <int D, int NS, bool A2>
+template <int D, int NS, int AM>
 int launch_bwd_col(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                    const CUtensorMap& mdo, const BwdParams& p, cudaStream_t st) {
-  auto kern = entmax_bwd_col_kernel<D, NS, A2>;
+  auto kern = entmax_bwd_col_kernel<D, NS, AM>;
   constexpr size_t smem = bwd_col_smem_bytes<D, NS>();
   static_assert(smem <= 232448, "bwd column kernel shared memory");
   static bool attr_ok = set_smem(kern, smem);
@@ -172,6 +174,48 @@ int launch_bwd_col(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.T);
   kern<<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
+}
+
+int alpha_mode(float alpha) {
+  return alpha == 2.0f ? AM_2 : (alpha == 1.5f ? AM_15 : AM_GEN);
+}
+
+// The forward kernel for this alpha and head dim (K/V ring depth 3 at D = 64, 2 at 128).
+template <int AM>
+int launch_fwd_d(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                 const FwdParams& p, cudaStream_t st) {
+  return D == 64 ? launch_fwd<64, 3, AM>(mq, mk, mv, p, st)
+                 : launch_fwd<128, 2, AM>(mq, mk, mv, p, st);
+}
+int launch_fwd_any(float alpha, int D, const CUtensorMap& mq, const CUtensorMap& mk,
+                   const CUtensorMap& mv, const FwdParams& p, cudaStream_t st) {
+  switch (alpha_mode(alpha)) {
+    case AM_2: return launch_fwd_d<AM_2>(D, mq, mk, mv, p, st);
+    case AM_15: return launch_fwd_d<AM_15>(D, mq, mk, mv, p, st);
+    default: return launch_fwd_d<AM_GEN>(D, mq, mk, mv, p, st);
+  }
+}
+
+// The backward row kernel, then the column kernel, for this alpha and head dim.
+template <int AM>
+int launch_bwd_d(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                 const CUtensorMap& mdo, const BwdParams& prow, const BwdParams& pcol,
+                 cudaStream_t st) {
+  int rc = D == 64 ? launch_bwd_row<64, 3, 2, AM>(mq, mk, mv, mdo, prow, st)
+                   : launch_bwd_row<128, 2, 2, AM>(mq, mk, mv, mdo, prow, st);
+  if (rc != ENTMAX_OK) return rc;
+  prof_mark(EV_BWD_ROW, st);
+  return D == 64 ? launch_bwd_col<64, 3, AM>(mq, mk, mv, mdo, pcol, st)
+                 : launch_bwd_col<128, 2, AM>(mq, mk, mv, mdo, pcol, st);
+}
+int launch_bwd_any(float alpha, int D, const CUtensorMap& mq, const CUtensorMap& mk,
+                   const CUtensorMap& mv, const CUtensorMap& mdo, const BwdParams& prow,
+                   const BwdParams& pcol, cudaStream_t st) {
+  switch (alpha_mode(alpha)) {
+    case AM_2: return launch_bwd_d<AM_2>(D, mq, mk, mv, mdo, prow, pcol, st);
+    case AM_15: return launch_bwd_d<AM_15>(D, mq, mk, mv, mdo, prow, pcol, st);
+    default: return launch_bwd_d<AM_GEN>(D, mq, mk, mv, mdo, prow, pcol, st);
+  }
 }
 
 // ------------------------------------------------------------ fixed scratch
@@ -326,13 +370,10 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
   p.vbar = reinterpret_cast<float*>(ws + L.vbar);
+  p.kpow = 1.0f / (alpha - 1.0f);
+  p.am1 = alpha - 1.0f;
 
-  const bool a2 = alpha == 2.0f;
-  if (D == 64) {
-    rc = a2 ? launch_fwd<64, 3, true>(mq, mk, mv, p, st) : launch_fwd<64, 3, false>(mq, mk, mv, p, st);
-  } else {
-    rc = a2 ? launch_fwd<128, 2, true>(mq, mk, mv, p, st) : launch_fwd<128, 2, false>(mq, mk, mv, p, st);
-  }
+  rc = launch_fwd_any(alpha, D, mq, mk, mv, p, st);
   prof_mark(EV_FWD1, st);
   return rc;
 }
@@ -390,11 +431,10 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, 
   p.inv_c_dn = std::nextafter(1.0f / p.c, 0.0f) * (1.0f - 1e-6f);
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.counters = reinterpret_cast<unsigned long long*>(ws + L.status + 8);
+  p.kpow = 1.0f / (alpha - 1.0f);
+  p.am1 = alpha - 1.0f;
 
-  const bool a2 = alpha == 2.0f;
-  if (D == 64)
-    return a2 ? launch_fwd<64, 3, true>(mq, mk, mv, p, st) : launch_fwd<64, 3, false>(mq, mk, mv, p, st);
-  return a2 ? launch_fwd<128, 2, true>(mq, mk, mv, p, st) : launch_fwd<128, 2, false>(mq, mk, mv, p, st);
+  return launch_fwd_any(alpha, D, mq, mk, mv, p, st);
 }
 
 int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
@@ -409,6 +449,10 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
       !aligned16(mask) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return ENTMAX_E_ALIGN;
+  // gradients only where g = p^(2 - alpha) is bounded (alpha <= 2): beyond, it
+  // is unbounded at the edge of the support and float32 scores cannot hold dQ,
+  // dK, dV to the bf16 tolerance
+  if (alpha > 2.0f) return ENTMAX_E_ALPHA;
   const WsLayout L = ws_layout(B, H, N, D, causal ? 1 : 0);
   if (workspace_bytes < L.total) return ENTMAX_E_WORKSPACE;
 
@@ -487,27 +531,13 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.status = status_word;
   p.counters = counters;
+  p.kpow = 1.0f / (alpha - 1.0f);
 
-  const bool a2 = alpha == 2.0f;
   BwdParams prow = p;
   prow.tm = tm;
   BwdParams pcol = p;
   pcol.tm = tmt;
-  if (D == 64) {
-    rc = a2 ? launch_bwd_row<64, 3, 2, true>(mq, mk, mv, mdo, prow, st)
-            : launch_bwd_row<64, 3, 2, false>(mq, mk, mv, mdo, prow, st);
-    if (rc != ENTMAX_OK) return rc;
-    prof_mark(EV_BWD_ROW, st);
-    rc = a2 ? launch_bwd_col<64, 3, true>(mq, mk, mv, mdo, pcol, st)
-            : launch_bwd_col<64, 3, false>(mq, mk, mv, mdo, pcol, st);
-  } else {
-    rc = a2 ? launch_bwd_row<128, 2, 2, true>(mq, mk, mv, mdo, prow, st)
-            : launch_bwd_row<128, 2, 2, false>(mq, mk, mv, mdo, prow, st);
-    if (rc != ENTMAX_OK) return rc;
-    prof_mark(EV_BWD_ROW, st);
-    rc = a2 ? launch_bwd_col<128, 2, true>(mq, mk, mv, mdo, pcol, st)
-            : launch_bwd_col<128, 2, false>(mq, mk, mv, mdo, pcol, st);
-  }
+  rc = launch_bwd_any(alpha, D, mq, mk, mv, mdo, prow, pcol, st);
   prof_mark(EV_BWD_COL, st);
   return rc;
 }
@@ -564,7 +594,7 @@ const char* entmax_attn_error_string(int code) {
     case ENTMAX_E_ALIGN: return "a tensor pointer is not 16-byte aligned (workspace: 256-byte)";
     case ENTMAX_E_SHAPE: return "B, H or N out of range";
     case ENTMAX_E_UNSUPPORTED: return "head dim, dtype or block size not supported";
-    case ENTMAX_E_ALPHA: return "alpha not supported (1.5 or 2.0)";
+    case ENTMAX_E_ALPHA: return "alpha outside [1.05, 3] (forward) or [1.05, 2] (backward)";
     case ENTMAX_E_WORKSPACE: return "workspace smaller than entmax_attn_workspace_size()";
     case ENTMAX_E_CUDA: return "a CUDA call failed";
     case ENTMAX_E_MAXITER: return "max_iter out of range";

@@ -50,6 +50,8 @@ struct FwdParams {
   __half* tmax;              // workspace: per-(row, key tile) maxima of s, rounded up
   float inv_c;               // 1 / c rounded up
   float inv_c_dn;            // 1 / c rounded down
+  float kpow;                // k = 1 / (alpha - 1): p = t^k, g = p^(2 - alpha) = t^(k - 1)
+  float am1;                 // alpha - 1
   uint32_t* status;          // workspace word 0
   unsigned long long* counters;  // workspace, CNT_* work counters
   // nullable, [BH][N][D]: g-weighted mean of v per row, sum_c g v_c / sum_c g
@@ -132,6 +134,94 @@ __device__ __forceinline__ float hist_lower_bound(const uint32_t (&cnt)[kNB + 1]
   }
   best += static_cast<float>(gtop - kNB) * (1.0f / kNB);
   return best - 2e-6f * fmaxf(1.0f, fabsf(best));
+}
+
+// tau_h for any alpha: bisection on the reduced problem sum_b c_b [x_b - tau]_+^k
+// = 1 over [x_top - 1, x_top] (x_top the highest non-empty lower edge; the
+// reduced function is >= 1 at its left end and 0 at its right), 20 halvings,
+// powers through pow_pos.  The left end of the final bracket, less 1e-4 for the
+// rounding of the powers, is returned (s-units): a lower bound of the exact root.
+__device__ __forceinline__ float hist_threshold_gen(const uint32_t (&cnt)[kNB + 1], int gtop,
+                                                    float k) {
+  int top = 0;
+#pragma unroll
+  for (int b = 0; b <= kNB; ++b) top = cnt[b] > 0u ? b : top;
+  float lo = static_cast<float>(top) * (1.0f / kNB) - 1.0f;
+  float hi = static_cast<float>(top) * (1.0f / kNB);
+#pragma unroll 1
+  for (int it = 0; it < 20; ++it) {
+    const float mid = 0.5f * (lo + hi);
+    float f = -1.0f;
+#pragma unroll
+    for (int b = 0; b <= kNB; ++b)
+      f = fmaf(static_cast<float>(cnt[b]), pow_pos(static_cast<float>(b) * (1.0f / kNB) - mid, k), f);
+    if (f > 0.0f) lo = mid;
+    else hi = mid;
+  }
+  return static_cast<float>(gtop - kNB) * (1.0f / kNB) + lo - 1e-4f;
+}
+
+// hist_lower_bound for any alpha: x_b - C_b^(-1/k), and for k >= 1 (x^k convex,
+// Jensen) min(x_b, mean_b - C_b^(-1/k)).  C^(-1/k) = 2^(-(alpha - 1) log2 C) is
+// inflated by 1e-5 for the rounding of the special-function unit.
+__device__ __forceinline__ float hist_lower_bound_gen(const uint32_t (&cnt)[kNB + 1], int gtop,
+                                                      float k, float am1) {
+  float best = -INFINITY;
+  uint32_t cc = 0u, aa = 0u;
+#pragma unroll
+  for (int b = kNB; b >= 0; --b) {
+    cc += cnt[b];
+    aa += cnt[b] * static_cast<uint32_t>(b);
+    const float cf = static_cast<float>(cc);
+    const float inv_k = exp2f(-am1 * __log2f(cf)) * 1.00001f;
+    const float xb = static_cast<float>(b) * (1.0f / kNB);
+    const float mean = static_cast<float>(aa) * (1.0f / kNB) / cf;
+    const float rb = k >= 1.0f ? fminf(xb, mean * 0.999998f - inv_k) : xb - inv_k;
+    best = cc > 0u ? fmaxf(best, rb) : best;
+  }
+  best += static_cast<float>(gtop - kNB) * (1.0f / kNB);
+  return best - 2e-6f * fmaxf(1.0f, fabsf(best));
+}
+
+// One safeguarded step for any alpha (zh §2.2, it §2B, ja §2.2, es §2B): Halley
+// for alpha <= 1.5, Newton beyond.  F0 = sum t^k, F1 = sum t^(k-1), F2 =
+// sum t^(k-2) over t = s - tau_c > 0; f = F0 - 1, f' = -k F1, f'' = k (k - 1) F2.
+// The Newton step solves the equivalent F0^(1/k) = 1 (the same root; for a
+// single support score it is linear in tau): tau + (F0^(1/k) - 1) F0 /
+// (F0^(1/k) F1).  The bracket [lo, hi] follows the sign of f; a step that
+// leaves it, or is longer than half the step taken two iterations earlier
+// (dx2; dx1 is the last one), is replaced by bisection, so the steps shrink
+// geometrically and no cycle survives.  Beyond alpha = 2 the pages take secant
+// steps; on the oracle this Newton step needs fewer (about 3.2 on average at
+// alpha = 3, against 5.0 for the secant, whose slowest rows had not converged
+// after 12).  Returns true once f is within 1e-4 and the step below
+// 1e-6 max(1, |tau|), or the bracket is that narrow -- the powers are accurate
+// to about 1e-6, so there is no exactness certificate as for the closed forms.
+__device__ __forceinline__ bool solver_step_gen(double F0, double F1, double F2, float k,
+                                                float& tau_c, double& lo, double& hi,
+                                                double& dx1, double& dx2) {
+  const double f = F0 - 1.0;
+  const double tc = tau_c;
+  if (f > 0.0) lo = fmax(lo, tc);
+  else if (f < 0.0) hi = fmin(hi, tc);
+  double tn = NAN;
+  if (k >= 2.0f) {
+    const double fp = -static_cast<double>(k) * F1;
+    const double fpp = static_cast<double>(k) * (k - 1.0f) * F2;
+    tn = tc - 2.0 * f * fp / (2.0 * fp * fp - f * fpp);          // Halley
+  } else if (F0 > 0.0 && F1 > 0.0) {
+    const double q = exp2(log2(F0) / static_cast<double>(k));     // F0^(1/k)
+    tn = tc + (q - 1.0) * F0 / (q * F1);                           // Newton on F0^(1/k)
+  }
+  if (!(tn > lo && tn < hi) || fabs(tn - tc) > 0.5 * fabs(dx2))
+    tn = 0.5 * (lo + hi);                                          // bisection fallback
+  dx2 = dx1;
+  dx1 = tn - tc;
+  const double tol = 1e-6 * fmax(1.0, fabs(tc));
+  const bool done =
+      f == 0.0 || (fabs(tn - tc) <= tol && fabs(f) <= 1e-4) || hi - lo <= 2.0 * tol;
+  tau_c = static_cast<float>(f == 0.0 ? tc : tn);
+  return done;
 }
 
 // Safety margin below tau_h that absorbs the rounding of s and tau (2^-20 |tau|).
@@ -272,11 +362,13 @@ __device__ __forceinline__ uint32_t hist_shifted(const uint32_t (&c)[kNB + 1], i
   return r;
 }
 
-template <int D, int NS, bool ALPHA2>
+template <int D, int NS, int AM>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     entmax_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const FwdParams P) {
+  constexpr bool ALPHA2 = AM == AM_2;
+  constexpr bool GEN = AM == AM_GEN;    // any other alpha: powers t^k
   extern __shared__ uint8_t smem_raw[];
   using Smem = FwdSmem<D, NS>;
   Smem& sm = *reinterpret_cast<Smem*>(align1024(smem_raw));
@@ -381,6 +473,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   int ncand1 = 0;                          // warpgroup 0: size of warpgroup 1's list
   double lo = 0.0, hi = 0.0;               // bracket of tau*
   double l_drop = -INFINITY;               // every score left out of the candidates is <= l_drop
+  double dx1 = INFINITY, dx2 = INFINITY;   // last two steps of the generic-alpha solver
   float tau_c = 0.0f;                      // current evaluation point / final tau
   int iter = 0;
   bool row_done = false;                   // threshold certified exact
@@ -625,7 +718,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           {
             acc_raw = fmaxf(acc_raw, __fsub_rd(m_raw, P.inv_c));
             if (row_ok && !cand_over && gtop_set && fmaxf(cmx0, cmx1) > acc_raw) {
-              const float lb = hist_lower_bound<ALPHA2>(cnt, gtop);   // s-units
+              const float lb = GEN ? hist_lower_bound_gen(cnt, gtop, P.kpow, P.am1)
+                                   : hist_lower_bound<ALPHA2>(cnt, gtop);   // s-units
               acc_raw = fmaxf(acc_raw, lb * (lb >= 0.0f ? P.inv_c_dn : P.inv_c));
             }
           }
@@ -713,7 +807,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               const float tp = fmaxf(tt, 0.0f);
               tmin[a] = in ? fminf(tmin[a], tt) : tmin[a];
               tneg[a] = in ? tneg[a] : fmaxf(tneg[a], tt);
-              if (ALPHA2) {
+              if (GEN) {
+                const float pk = pow_pos(tt, P.kpow);
+                const float pk1 = in ? __fdividef(pk, tt) : 0.0f;     // t^(k-1)
+                f0[a] += pk;
+                f1[a] += pk1;
+                if (P.kpow >= 2.0f) f2[a] += in ? __fdividef(pk1, tt) : 0.0f;
+              } else if (ALPHA2) {
                 f0[a] += tp;
                 f1[a] += in ? 1.0f : 0.0f;
               } else {
@@ -751,11 +851,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int e = 0; e < 16; ++e) {
               const float t0 = fmaxf(fmaf(v[2 * e], P.c, -tau_c), 0.0f);
               const float t1 = fmaxf(fmaf(v[2 * e + 1], P.c, -tau_c), 0.0f);
-              const float p0 = ALPHA2 ? t0 : t0 * t0;
-              const float p1 = ALPHA2 ? t1 : t1 * t1;
-              // g = p^(2 - alpha): the support indicator at alpha = 2, t at 1.5
-              const float g0 = ALPHA2 ? (t0 > 0.0f ? 1.0f : 0.0f) : t0;
-              const float g1 = ALPHA2 ? (t1 > 0.0f ? 1.0f : 0.0f) : t1;
+              float p0, p1, g0, g1;
+              if (GEN) {
+                // g = t^(k - 1), held below 6e4 (fp16) where alpha > 2 lets it grow
+                // without bound at the edge of the support
+                p0 = pow_pos(t0, P.kpow);
+                p1 = pow_pos(t1, P.kpow);
+                g0 = t0 > 0.0f ? fminf(__fdividef(p0, t0), 6.0e4f) : 0.0f;
+                g1 = t1 > 0.0f ? fminf(__fdividef(p1, t1), 6.0e4f) : 0.0f;
+              } else {
+                p0 = ALPHA2 ? t0 : t0 * t0;
+                p1 = ALPHA2 ? t1 : t1 * t1;
+                // g = p^(2 - alpha): the support indicator at alpha = 2, t at 1.5
+                g0 = ALPHA2 ? (t0 > 0.0f ? 1.0f : 0.0f) : t0;
+                g1 = ALPHA2 ? (t1 > 0.0f ? 1.0f : 0.0f) : t1;
+              }
               ps[e & 3] += p0 + p1;
               gs[e & 3] += g0 + g1;
               if (gv) {
@@ -855,7 +965,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               const float tp = fmaxf(tt, 0.0f);
               tmn[a] = in ? fminf(tmn[a], tt) : tmn[a];
               tng[a] = in ? tng[a] : fmaxf(tng[a], tt);
-              if (ALPHA2) {
+              if (GEN) {
+                const float pk = pow_pos(tt, P.kpow);
+                const float pk1 = in ? __fdividef(pk, tt) : 0.0f;     // t^(k-1)
+                f0[a] += pk;
+                f1[a] += pk1;
+                if (P.kpow >= 2.0f) f2[a] += in ? __fdividef(pk1, tt) : 0.0f;
+              } else if (ALPHA2) {
                 f0[a] += tp;
                 f1[a] += in ? 1.0f : 0.0f;
               } else {
@@ -870,7 +986,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const double F2c = (f2[0] + f2[1]) + (f2[2] + f2[3]);
           const float tminc = fminf(fminf(tmn[0], tmn[1]), fminf(tmn[2], tmn[3]));
           const float tnegc = fmaxf(fmaxf(tng[0], tng[1]), fmaxf(tng[2], tng[3]));
-          row_done = solver_step<ALPHA2>(F0c, F1c, F2c, tminc, tnegc, l_drop, tau_c, lo, hi);
+          row_done = GEN ? solver_step_gen(F0c, F1c, F2c, P.kpow, tau_c, lo, hi, dx1, dx2)
+                         : solver_step<ALPHA2>(F0c, F1c, F2c, tminc, tnegc, l_drop, tau_c, lo, hi);
           ++iter;
           trace_store(iter, tau_c);
         }
@@ -951,10 +1068,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ncand1 = x.ncand;
           cand_over = cand_over || x.over;
           if (fabsf(m_raw * P.cN) >= 2097152.0f) atomicOr(P.status, ST_RANGE);
-          tau_h = hist_threshold<ALPHA2>(cnt, gtop);
+          tau_h = GEN ? static_cast<double>(hist_threshold_gen(cnt, gtop, P.kpow))
+                      : hist_threshold<ALPHA2>(cnt, gtop);
           const double margin = hist_margin(tau_h);
           const double m_s = static_cast<double>(m_raw) * P.c;
-          const double nb = ALPHA2 ? 1.0 / n_valid : 1.0 / sqrt(static_cast<double>(n_valid));
+          // n^(1 - alpha), the distance of tau* below the max at the latest
+          const double nb =
+              GEN ? static_cast<double>(exp2f(-P.am1 * __log2f(static_cast<float>(n_valid)))) *
+                        (1.0 - 1e-5)
+                  : (ALPHA2 ? 1.0 / n_valid : 1.0 / sqrt(static_cast<double>(n_valid)));
           lo = tau_h - margin;
           hi = fmin(tau_h + 1.0 / kNB + margin, m_s - nb + margin);
           l_drop = static_cast<double>(acc_raw) * P.c;   // every unlisted score is <= l_drop <= tau*
@@ -1011,7 +1133,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           F2 += sm.xf[2][rl];
           Tmin = fminf(Tmin, sm.xtmin[rl]);
           Tneg = fmaxf(Tneg, sm.xtneg[rl]);
-          row_done = solver_step<ALPHA2>(F0, F1, F2, Tmin, Tneg, l_drop, tau_c, lo, hi);
+          row_done = GEN ? solver_step_gen(F0, F1, F2, P.kpow, tau_c, lo, hi, dx1, dx2)
+                         : solver_step<ALPHA2>(F0, F1, F2, Tmin, Tneg, l_drop, tau_c, lo, hi);
           ++iter;
           trace_store(iter, tau_c);
           if (!row_done && iter < P.max_iter) sm.not_converged = 1;
@@ -1082,7 +1205,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (wg == 0 && row_ok) {
           rowsum += sm.xsum[rl];
           P.tau[static_cast<size_t>(bh) * P.N + row] = tau_c;
-          if (!(fabsf(rowsum - 1.0f) <= 1e-3f)) atomicOr(P.status, ST_NOT_CONVERGED);
+          // sum p = 1 within 1e-3; for k < 1 (alpha > 2) p = t^k turns a rounding
+          // eps of s or tau (2^-23 of their magnitude) into eps^k at the edge of
+          // the support, so the check allows 8 such terms
+          float sum_tol = 1e-3f;
+          if (GEN && P.kpow < 1.0f)
+            sum_tol = fmaxf(sum_tol, 8.0f * pow_pos(1.2e-7f * (fabsf(tau_c) + 2.0f), P.kpow));
+          if (!(fabsf(rowsum - 1.0f) <= sum_tol)) atomicOr(P.status, ST_NOT_CONVERGED);
         }
         if (wg == 0)
           for (int it = iter + 1; it <= P.max_iter; ++it) trace_store(it, tau_c);

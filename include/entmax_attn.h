@@ -15,7 +15,7 @@
  * How (zh §2.1-2.3, it §2A-2C, ja §2.1-2.3, es §2A-2C): one streaming pass
  * over the key blocks builds an on-chip histogram of the scores per query row
  * and solves the reduced problem for a lower bound tau_h of tau; one or two
- * safeguarded Halley (alpha = 1.5) or Newton (alpha = 2) steps refine it; a
+ * safeguarded Halley (alpha <= 1.5) or Newton (beyond) steps refine it; a
  * bit-packed block mask (32 blocks per uint32) records the non-zero blocks and
  * P.V, dQ, dK and dV visit only those blocks.
  *
@@ -37,8 +37,10 @@
  *     1 within 1e-3, a bounded wait that timed out, an out-of-range score) are
  *     OR-ed into a status word at the start of the workspace; read it with
  *     entmax_attn_status().  Kernels never trap.
- *   - Supported: D in {64, 128}; block in {64, 128}; alpha in {1.5, 2.0};
- *     1 <= N <= ENTMAX_MAX_N; dtype bf16 (tcgen05 tensor-core path) or fp32
+ *   - Supported: D in {64, 128}; block in {64, 128}; 1 <= N <= ENTMAX_MAX_N;
+ *     alpha in [1.05, 3] for bf16 (closed forms at 1.5 and 2, powers
+ *     t^(1/(alpha-1)) through the special-function unit otherwise) and
+ *     {1.5, 2.0} for fp32; dtype bf16 (tcgen05 tensor-core path) or fp32
  *     (CUDA-core path for full fp32 precision, D = 64 only).
  */
 #ifndef ENTMAX_ATTN_H
@@ -57,7 +59,7 @@ extern "C" {
 #define ENTMAX_E_ALIGN       -2  /* a tensor pointer is not 16-byte aligned         */
 #define ENTMAX_E_SHAPE       -3  /* B, H or N out of range                          */
 #define ENTMAX_E_UNSUPPORTED -4  /* D, dtype or block not supported                 */
-#define ENTMAX_E_ALPHA       -5  /* alpha not supported                             */
+#define ENTMAX_E_ALPHA       -5  /* alpha outside [1.05, 3]                         */
 #define ENTMAX_E_WORKSPACE   -6  /* workspace smaller than entmax_attn_workspace_size */
 #define ENTMAX_E_CUDA        -7  /* a CUDA call failed (launch, tensor-map encode)  */
 #define ENTMAX_E_MAXITER     -8  /* max_iter outside [0, ENTMAX_MAX_ITER]            */
@@ -74,7 +76,7 @@ extern "C" {
 #define ENTMAX_ST_RANGE         4u /* |s| * 8 reached 2^21 somewhere: histogram inexact */
 
 #define ENTMAX_MAX_N    262144
-#define ENTMAX_MAX_ITER 8
+#define ENTMAX_MAX_ITER 16
 #define ENTMAX_NOALLOC_SCRATCH_BYTES (8u << 20)
 
 /*
@@ -101,7 +103,18 @@ size_t entmax_attn_workspace_size(int B, int H, int N, int D, int block, int cau
  * skipping); it §2A-2C; ja §2.1-2.3; es §2A-2C.
  *
  *   q, k, v      in   [B][H][N][D], dtype.
- *   alpha        in   1.5 (Halley steps) or 2.0 (Newton steps).
+ *   alpha        in   in [1.05, 3].  1.5 and 2.0 use closed forms (p = t^2, p = t)
+ *                     and certified-exact Halley / Newton steps; any other alpha
+ *                     computes p = t^(1/(alpha-1)) with the special-function unit
+ *                     (relative error about 1e-6) and takes Halley (alpha < 1.5)
+ *                     or Newton steps, bisection-safeguarded, until f is within
+ *                     1e-4 and the step below 1e-6 max(1, |tau|) (zh §2.2,
+ *                     es §2B); give it a max_iter of about 12.  Beyond alpha = 3
+ *                     a float32 tau cannot hold the outputs to 2e-2: p = t^k has
+ *                     an unbounded slope where a score enters the support.  For
+ *                     alpha > 2, g = p^(2-alpha) also grows without bound there:
+ *                     the forward holds g below 6e4 in the G.V product, and
+ *                     entmax_attn_bwd rejects alpha > 2.
  *   causal       in   nonzero: key c is visible to query r iff c <= r.
  *   block        in   block size of the mask (64 or 128), rows and keys alike.
  *   max_iter     in   at most this many refinement passes after the histogram
@@ -172,7 +185,10 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, 
  *
  *   q, k, v, dout  in  [B][H][N][D], dtype.
  *   tau, mask      in  exactly as written by entmax_attn_fwd for these inputs.
- *   alpha, causal, block   as given to entmax_attn_fwd.
+ *   alpha, causal, block   as given to entmax_attn_fwd; alpha in [1.05, 2]
+ *                  (ENTMAX_E_ALPHA beyond: g = p^(2-alpha) is unbounded at the
+ *                  edge of the support, where float32 scores cannot hold the
+ *                  gradients to the bf16 tolerance -- 0.14 on dQ at alpha = 3).
  *   dq, dk, dv     out [B][H][N][D], dtype (fully overwritten).
  *   workspace      in/out  the same size rule as for the forward; status bits
  *                  are OR-ed into the existing status word.  bf16: the

@@ -66,9 +66,12 @@ def test_forward_argument_validation(lib):
     assert fwd(lib, dtype=7) == dsa.E_UNSUPPORTED
     assert fwd(lib, dtype=1, D=128) == dsa.E_UNSUPPORTED   # fp32 path: head dim 64
     assert fwd(lib, alpha=1.0) == dsa.E_ALPHA
-    assert fwd(lib, alpha=1.7) == dsa.E_ALPHA
+    assert fwd(lib, alpha=1.02) == dsa.E_ALPHA    # k = 1/(alpha - 1) above 20
+    assert fwd(lib, alpha=3.5) == dsa.E_ALPHA
+    assert fwd(lib, alpha=float("nan")) == dsa.E_ALPHA
+    assert fwd(lib, dtype=1, alpha=1.7) == dsa.E_UNSUPPORTED   # fp32 path: 1.5 and 2 only
     assert fwd(lib, max_iter=-1) == dsa.E_MAXITER
-    assert fwd(lib, max_iter=9) == dsa.E_MAXITER
+    assert fwd(lib, max_iter=17) == dsa.E_MAXITER
     assert fwd(lib, q=MISALIGNED) == dsa.E_ALIGN
     assert fwd(lib, ws_bytes=1) == dsa.E_WORKSPACE
 
@@ -82,7 +85,9 @@ def test_backward_argument_validation(lib):
     assert bwd(q=None) == dsa.E_NULL
     assert bwd(dq=None) == dsa.E_NULL
     assert bwd(D=32) == dsa.E_UNSUPPORTED
-    assert bwd(alpha=3.0) == dsa.E_ALPHA
+    assert bwd(alpha=5.0) == dsa.E_ALPHA
+    assert bwd(alpha=2.5) == dsa.E_ALPHA     # gradients: alpha <= 2 only
+    assert bwd(alpha=1.75, q=None) == dsa.E_NULL   # generic alpha <= 2 is accepted
     assert bwd(q=MISALIGNED) == dsa.E_ALIGN
     assert bwd(ws_bytes=0) == dsa.E_WORKSPACE
 

@@ -113,7 +113,7 @@ def test_t3_t4_row_sums_and_bounds(alpha):
 
 @pytest.mark.parametrize("anchor", ["grid", "max"])
 @pytest.mark.parametrize("n_bins", [8, 16, 32])
-@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 3.0])
 def test_t5_histogram_lower_bound(anchor, n_bins, alpha):
     """Proposition 1 as the summaries state it (zh §2.1, ja §2.1):
     tau* - h < tau_h <= tau*, and the support at tau_h contains the true one
@@ -168,7 +168,7 @@ def test_t6_jacobian_finite_differences(alpha):
         np.testing.assert_allclose(O.entmax_jvp(p, v, alpha), fd, rtol=0, atol=1e-7)
 
 
-@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.3, 3.0])
 @pytest.mark.parametrize("causal", [True, False])
 def test_t6_attention_gradients_finite_differences(alpha, causal):
     """dQ, dK, dV against central differences of L = <O, dO>."""

@@ -9,9 +9,12 @@ fallback; the two share no code.
 
 Citations name the gist.science summary pages of "AdaSplash-2: Faster
 Differentiable Sparse Attention" by their language (zh, it, ja, es) and the
-section on that page.
+section on that page.  ``dash_router`` covers the stage-0/1 router of
+DashAttention from the Italian summary of that paper, which the same pages
+carry.
 """
 
+from . import dash_router  # noqa: F401
 from .entmax_oracle import (  # noqa: F401
     attention_backward,
     attention_forward,

@@ -28,6 +28,9 @@ EXPORTED = ("entmax_attn_mask_words", "entmax_attn_workspace_size", "entmax_attn
             "entmax_attn_bwd", "entmax_attn_status", "entmax_attn_counters",
             "entmax_attn_profile", "entmax_attn_profile_read", "entmax_attn_error_string",
             "entmax_attn_fwd_noalloc")
+# include/dash_route.h: the DashAttention stage-0/1 router
+DASH_EXPORTED = ("dash_route_workspace_size", "dash_route_fwd")
+DASH_MAX_CHUNKS = 256
 COUNTER_NAMES = ("fwd_hist_tiles", "fwd_refine_tiles", "fwd_pv_tiles", "fwd_refine_passes",
                  "bwd_row_tiles", "bwd_col_tiles", "fwd_cand_overflow_tiles")
 PHASE_NAMES = ("fwd", "bwd_fp16_copies", "bwd_tile_masks", "bwd_row", "bwd_col")
@@ -75,6 +78,11 @@ def _lib():
     lib.entmax_attn_fwd_noalloc.restype = c_int
     lib.entmax_attn_error_string.argtypes = [c_int]
     lib.entmax_attn_error_string.restype = ctypes.c_char_p
+    lib.dash_route_workspace_size.argtypes = [c_int] * 6
+    lib.dash_route_workspace_size.restype = c_size
+    lib.dash_route_fwd.argtypes = ([vp, vp] + [c_int] * 6 + [c_float, c_float, c_int]
+                                   + [vp] * 4 + [c_size, vp])
+    lib.dash_route_fwd.restype = c_int
     _lib_handle = lib
     return lib
 
@@ -242,3 +250,43 @@ class EntmaxAttention(torch.autograd.Function):
 
 def entmax_attention(q, k, v, alpha=1.5, causal=True, block=128, max_iter=None):
     return EntmaxAttention.apply(q, k, v, alpha, causal, block, max_iter)
+
+
+# ------------------------------------------------------------------ DashAttention router
+class RouteResult(NamedTuple):
+    wbar: torch.Tensor        # float32 [B, Hkv, N, C]
+    row_mask: torch.Tensor    # int32 (uint32 bits) [B, Hkv, N, ceil(C / 32)]
+    block_mask: torch.Tensor  # int32 (uint32 bits) [B, Hkv, ceil(N / 128), ceil(C / 32)]
+    workspace: torch.Tensor
+
+
+def dash_route(q, k, chunk: int, gamma: float, alpha: float = 1.5, max_iter=None, *,
+               stream=None) -> RouteResult:
+    """DashAttention stages 0-1 through ``dash_route_fwd``: chunk-mean summaries
+    of k, alpha-entmax routing of every query row over the complete chunks
+    before its own, averaged over the query heads of each KV head (GQA).
+    q: [B, Hq, N, D] bf16, k: [B, Hkv, N, D] bf16, Hq a multiple of Hkv."""
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
+        raise TypeError("dash_route: q and k must be bfloat16")
+    if not (q.is_cuda and k.is_cuda and q.is_contiguous() and k.is_contiguous()):
+        raise ValueError("dash_route: q and k must be contiguous CUDA tensors")
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, D):
+        raise ValueError("dash_route: k must be [B, Hkv, N, D] with q's B, N and D")
+    max_iter = default_max_iter(alpha) if max_iter is None else int(max_iter)
+    dev = q.device
+    C = N // int(chunk)
+    W = (C + 31) // 32
+    wbar = torch.empty((B, Hkv, N, C), dtype=torch.float32, device=dev)
+    row_mask = torch.empty((B, Hkv, N, W), dtype=torch.int32, device=dev)
+    block_mask = torch.empty((B, Hkv, (N + 127) // 128, W), dtype=torch.int32, device=dev)
+    ws_bytes = int(_lib().dash_route_workspace_size(B, Hq, Hkv, N, D, int(chunk)))
+    workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    rc = _lib().dash_route_fwd(
+        _ptr(q), _ptr(k), B, Hq, Hkv, N, D, int(chunk), float(gamma), float(alpha), max_iter,
+        _ptr(wbar), _ptr(row_mask), _ptr(block_mask), _ptr(workspace), ws_bytes,
+        _stream_ptr(stream, dev))
+    if rc != OK:
+        raise EntmaxError(rc, "dash_route_fwd")
+    return RouteResult(wbar, row_mask, block_mask, workspace)

@@ -12,6 +12,8 @@
 #include <mutex>
 
 #include "entmax_attn.h"
+#include "dash_route.h"
+#include "dash.cuh"
 #include "fwd.cuh"
 #include "bwd.cuh"
 #include "simt32.cuh"
@@ -286,6 +288,51 @@ int launch_bwd_f32(const F32Params& p, cudaStream_t st) {
 }  // namespace
 
 // ============================================================== C ABI
+// ------------------------------------------------------- DashAttention router
+namespace {
+struct DashLayout {
+  size_t status = 0, kbar = 0, q16 = 0, total = 0;
+  int C = 0, Cp = 0;
+};
+DashLayout dash_layout(int B, int Hq, int Hkv, int N, int D, int chunk) {
+  DashLayout L;
+  L.C = N / chunk;
+  L.Cp = (L.C + kTile - 1) / kTile * kTile;
+  size_t off = 256;
+  L.kbar = off;
+  off = align256(off + 2 * static_cast<size_t>(B) * Hkv * L.Cp * D * sizeof(__half));
+  L.q16 = off;
+  off = align256(off + static_cast<size_t>(B) * Hq * N * D * sizeof(__half));
+  L.total = off;
+  return L;
+}
+int dash_check(int B, int Hq, int Hkv, int N, int D, int chunk) {
+  if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || N < 1 || N > kMaxN || chunk < 1)
+    return ENTMAX_E_SHAPE;
+  if (N / chunk > DASH_MAX_CHUNKS) return ENTMAX_E_SHAPE;
+  if (static_cast<long long>(B) * Hkv * ((N + kTile - 1) / kTile) > 0x7fffffffLL) return ENTMAX_E_SHAPE;
+  if (D != 64 && D != 128) return ENTMAX_E_UNSUPPORTED;
+  return ENTMAX_OK;
+}
+template <int D, int AM>
+int launch_dash(const CUtensorMap& mq, const CUtensorMap& mkb, const DashParams& p,
+                cudaStream_t st) {
+  auto kern = dash_route_kernel<D, AM>;
+  constexpr size_t smem = dash_smem_bytes<D>();
+  static_assert(smem <= 232448, "router kernel shared memory");
+  static bool attr_ok = set_smem(kern, smem);
+  if (!attr_ok) return ENTMAX_E_CUDA;
+  const unsigned grid = static_cast<unsigned>(p.BHkv) * static_cast<unsigned>(p.tr);
+  kern<<<grid, kDashThreads, smem, st>>>(mq, mkb, p);
+  return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
+}
+template <int AM>
+int launch_dash_d(int D, const CUtensorMap& mq, const CUtensorMap& mkb, const DashParams& p,
+                  cudaStream_t st) {
+  return D == 64 ? launch_dash<64, AM>(mq, mkb, p, st) : launch_dash<128, AM>(mq, mkb, p, st);
+}
+}  // namespace
+
 extern "C" {
 
 int entmax_attn_mask_words(int N, int block) {
@@ -585,6 +632,75 @@ int entmax_attn_profile_read(float* ms, int n) {
       return ENTMAX_E_CUDA;
   }
   return ENTMAX_OK;
+}
+
+
+size_t dash_route_workspace_size(int B, int Hq, int Hkv, int N, int D, int chunk) {
+  if (dash_check(B, Hq, Hkv, N, D, chunk) != ENTMAX_OK) return 0;
+  return dash_layout(B, Hq, Hkv, N, D, chunk).total;
+}
+
+int dash_route_fwd(const void* q, const void* k, int B, int Hq, int Hkv, int N, int D, int chunk,
+                   float gamma, float alpha, int max_iter, float* wbar, uint32_t* row_mask,
+                   uint32_t* block_mask, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !workspace) return ENTMAX_E_NULL;
+  int rc = dash_check(B, Hq, Hkv, N, D, chunk);
+  if (rc != ENTMAX_OK) return rc;
+  if (N / chunk == 0) return ENTMAX_OK;   // no complete chunk: the outputs are empty
+  if (!wbar || !row_mask || !block_mask) return ENTMAX_E_NULL;
+  if (!(alpha >= 1.05f && alpha <= 3.0f)) return ENTMAX_E_ALPHA;
+  if (!(gamma > 0.0f) || !std::isfinite(gamma)) return ENTMAX_E_SHAPE;
+  if (max_iter < 0 || max_iter > ENTMAX_MAX_ITER) return ENTMAX_E_MAXITER;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(wbar) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(row_mask) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(block_mask) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return ENTMAX_E_ALIGN;
+  const DashLayout L = dash_layout(B, Hq, Hkv, N, D, chunk);
+  if (workspace_bytes < L.total) return ENTMAX_E_WORKSPACE;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  if (cudaMemsetAsync(ws + L.status, 0, 256, st) != cudaSuccess) return ENTMAX_E_CUDA;
+  __half* q16 = reinterpret_cast<__half*>(ws + L.q16);
+  __half* kbar = reinterpret_cast<__half*>(ws + L.kbar);
+  launch_to_fp16(static_cast<const __nv_bfloat16*>(q), q16, static_cast<size_t>(B) * Hq * N * D,
+                 status, st);
+  {
+    const long long total = static_cast<long long>(B) * Hkv * L.Cp * (D / 8);
+    const int grid = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 8));
+    dash_chunk_mean_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k), kbar, B * Hkv,
+                                                 N, D, chunk, L.C, L.Cp);
+  }
+  if (cudaGetLastError() != cudaSuccess) return ENTMAX_E_CUDA;
+  CUtensorMap mq, mkb;
+  const auto f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  if (!make_map(&mq, q16, B * Hq, N, D, f16) || !make_map(&mkb, kbar, 2 * B * Hkv, L.Cp, D, f16))
+    return ENTMAX_E_CUDA;
+
+  DashParams p{};
+  p.BHkv = B * Hkv;
+  p.G = Hq / Hkv;
+  p.N = N;
+  p.C = L.C;
+  p.Cp = L.Cp;
+  p.chunk = chunk;
+  p.tr = (N + kTile - 1) / kTile;
+  p.max_iter = max_iter;
+  p.c = (alpha - 1.0f) * gamma / std::sqrt(static_cast<float>(D));
+  p.kpow = 1.0f / (alpha - 1.0f);
+  p.am1 = alpha - 1.0f;
+  p.wbar = wbar;
+  p.row_mask = row_mask;
+  p.block_mask = block_mask;
+  p.W = (L.C + 31) / 32;
+  p.status = status;
+  switch (alpha_mode(alpha)) {
+    case AM_2: return launch_dash_d<AM_2>(D, mq, mkb, p, st);
+    case AM_15: return launch_dash_d<AM_15>(D, mq, mkb, p, st);
+    default: return launch_dash_d<AM_GEN>(D, mq, mkb, p, st);
+  }
 }
 
 const char* entmax_attn_error_string(int code) {

@@ -12,6 +12,8 @@ Workloads (seeded synthetic data, see differentiable_sparse_attention_b200/workl
   sparsemax_16k   B=1 H=16 N=16384 D=128 alpha=2 t=3
   planted_32k     B=1 H=8 N=32768 D=128 alpha=1.5, 32 planted key blocks per head
   long_sweep      B=1 H=8 D=128 t=4, alpha in {1.5, 2}, N in {65536, 131072}
+  dash_router_16k DashAttention stage-0/1 router: B=1, 32 query heads over 8 KV heads,
+                  N=16384 D=128, chunks of 64 (256 chunks), gamma=16, alpha=1.5
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (the
 (batch, head) problems are independent: weak scaling, no collective on the
@@ -438,6 +440,117 @@ def run_reference(args, points, rank, world):
     }
 
 
+ROUTER = dict(B=1, Hq=32, Hkv=8, N=16384, D=128, chunk=64, gamma=16.0, alpha=1.5, seed=0)
+
+
+def run_router(args, rank, world, device):
+    """One step = dash_route on seeded N(0,1) bf16 q and k of the router
+    workload.  value = logit FLOPs (2 B Hq N C D, one GEMM) per second; the
+    roofline counts the MMAs the kernel issues (two fp16 parts of the chunk
+    summaries over 128-row and 128-chunk tiles) against the call's event time,
+    which also covers the fp16 copy of q and the chunk means."""
+    import differentiable_sparse_attention_b200 as dsa
+
+    w = dict(ROUTER)
+    if args.alpha:
+        w["alpha"] = args.alpha
+    peaks, peaks_kind = load_peaks()
+    g = torch.Generator().manual_seed(w["seed"])
+    qh = torch.randn((w["B"], w["Hq"], w["N"], w["D"]), generator=g).to(torch.bfloat16)
+    kh = torch.randn((w["B"], w["Hkv"], w["N"], w["D"]), generator=g).to(torch.bfloat16)
+    q, k = qh.to(device), kh.to(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    step = lambda: dsa.dash_route(q, k, w["chunk"], w["gamma"], w["alpha"])
+    for _ in range(max(3, args.warmup)):
+        res = step()
+    torch.cuda.synchronize(device)
+    st = dsa.status(res.workspace)
+    C = w["N"] // w["chunk"]
+    active = res.wbar > 0
+    density = float(active[..., w["chunk"]:, :].float().mean().item())
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    ms = []
+    with ClockSampler(device.index) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            ev0.record()
+            res = step()
+            ev1.record()
+            ev1.synchronize()
+            ms.append(ev0.elapsed_time(ev1))
+    ms_sum = max_over_ranks(sum(ms), device)
+    ms_step = ms_sum / args.steps
+    logit_flop = 2.0 * w["B"] * w["Hq"] * w["N"] * C * w["D"]
+    value = logit_flop * world / (ms_step * 1e-3) / 1e12
+    tr = (w["N"] + 127) // 128
+    cp = (C + 127) // 128 * 128
+    mma_flop = 2 * 2.0 * w["B"] * w["Hq"] * tr * 128 * cp * w["D"]
+    achieved = mma_flop / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": "DashAttention stage-1 entmax router ms/call & logit TFLOP/s, 1 B200",
+        "value": round(value, 3), "unit": "logit TFLOP/s (2*B*Hq*N*C*D per call)",
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) q, k)",
+        "config": {"workload": "dash_router_16k: " + ", ".join(f"{a}={b}" for a, b in w.items()),
+                   "l2": "flushed (256 MB write) before every step",
+                   "parallelism": f"replica x{world}"},
+        "chunk_density": round(density, 4), "status": st,
+        "roofline": {"bound": "tensor", "kernel": "dash_route (whole call)",
+                     "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "traffic": None,
+                     "note": f"issued MMA FLOPs / call time (fp16 copy of q and chunk means "
+                             f"included); peak = {peaks_kind} dense bf16 burst"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+def run_router_reference(args, world):
+    """The router oracle on the host cores: each step routes 128 evenly spread
+    query rows of KV head 0 (its 4 query heads) of the router workload."""
+    from oracle import dash_router as R
+
+    w = dict(ROUTER)
+    if args.alpha:
+        w["alpha"] = args.alpha
+    g = torch.Generator().manual_seed(w["seed"])
+    qh = torch.randn((w["B"], w["Hq"], w["N"], w["D"]), generator=g).to(torch.bfloat16)
+    kh = torch.randn((w["B"], w["Hkv"], w["N"], w["D"]), generator=g).to(torch.bfloat16)
+    G = w["Hq"] // w["Hkv"]
+    q64 = qh[0, :G].double().numpy()
+    k64 = kh[0, :1].double().numpy()
+    rows = np.unique(np.linspace(0, w["N"] - 1, 128).round().astype(np.int64))
+    C = w["N"] // w["chunk"]
+    r0 = resource.getrusage(resource.RUSAGE_SELF)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        R.route(q64, k64, w["alpha"], w["gamma"], w["chunk"], rows=rows)
+    wall = time.perf_counter() - t0
+    r1 = resource.getrusage(resource.RUSAGE_SELF)
+    cores = max(1, round(((r1.ru_utime - r0.ru_utime) + (r1.ru_stime - r0.ru_stime)) / wall))
+    flop = 2.0 * G * rows.size * C * w["D"] * args.steps
+    value = flop / wall / 1e12
+    sample = (f"{rows.size} evenly spread rows x {G} query heads of KV head 0 per step "
+              f"({args.steps} steps, {wall:.1f} s)")
+    return {"impl": "reference",
+            "metric": "DashAttention stage-1 entmax router ms/call & logit TFLOP/s, 1 B200",
+            "value": round(value, 8), "unit": "logit TFLOP/s (2*B*Hq*N*C*D per call)",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(wall * 1e3 / args.steps, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "dash_router_16k (oracle sample)", "sample": sample},
+            "cpu_baseline": {"value": round(value, 8), "unit": "logit TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 8), "unit": "logit TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -452,6 +565,26 @@ def main():
     ap.add_argument("--alpha", type=float, default=0.0,
                     help="override alpha (any value in [1.05, 3]; 1.5 and 2 have closed forms)")
     args = ap.parse_args()
+    if args.workload == "dash_router_16k":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps(run_router_reference(args, world)))
+            return
+        device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+        torch.cuda.set_device(device)
+        if world > 1:
+            import datetime
+            torch.distributed.init_process_group("nccl", device_id=device,
+                                                 timeout=datetime.timedelta(seconds=120))
+        line = run_router(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(line))
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     points = workload_points(args.workload)
     if args.heads:
         points = [p.with_(H=args.heads) for p in points]

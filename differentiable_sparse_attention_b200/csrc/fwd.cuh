@@ -303,9 +303,10 @@ struct FwdSmem {
   __nv_bfloat16 q[kTile * D];       // D/64 swizzled slabs
   __nv_bfloat16 k[NS][kTile * D];
   __nv_bfloat16 v[NS][kTile * D];
-  // candidate storage beyond the V ring (P and G of the P.V pass live in TMEM)
-  static constexpr int kNSP = D == 64 ? 2 : 1;
-  __nv_bfloat16 p[kNSP][kTile * kTile];
+  // candidate storage beyond the V ring (P and G of the P.V pass live in TMEM),
+  // in slots of one float per row: what the 227 KB of shared memory leave
+  static constexpr int kCandXSlots = D == 64 ? 184 : 88;
+  float cx[kCandXSlots * kTile];
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS];
   uint64_t v_full[NS], v_empty[NS];
@@ -329,16 +330,16 @@ struct FwdSmem {
   int xflag[kTile];           // 0 -> 1: list rebuilt by COLLECT
 };
 
-// Candidate scores live in the V ring and the P tiles, which stay idle until
-// the P.V pass: slot-major [cap][128 rows] floats (thread r uses column r, so
+// Candidate scores live in the V ring and the slots after it, which stay idle
+// until the P.V pass: slot-major [cap][128 rows] floats (thread r uses column r, so
 // appends and reads are free of bank conflicts); warpgroup h owns slots
 // [h cap/2, (h + 1) cap/2).  A list is compacted at most kMaxPrunes times;
 // after that it is rebuilt by a COLLECT pass.
-constexpr int kMaxPrunes = 8;
+constexpr int kMaxPrunes = 16;
 
 template <int D, int NS>
 __host__ __device__ constexpr int fwd_cand_cap() {
-  return (NS * kTile * D * 2 + FwdSmem<D, NS>::kNSP * kTile * kTile * 2) / (4 * kTile);
+  return (NS * kTile * D * 2) / (4 * kTile) + FwdSmem<D, NS>::kCandXSlots;
 }
 
 template <int D, int NS>
@@ -383,8 +384,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   constexpr uint32_t kColG = 256 + D;
   constexpr int kCap = fwd_cand_cap<D, NS>();
   constexpr int kCapH = kCap / 2;
-  static_assert(offsetof(Smem, p) == offsetof(Smem, v) + NS * kTile * D * 2,
-                "candidates need the V ring and the P tiles to be adjacent");
+  static_assert(offsetof(Smem, cx) == offsetof(Smem, v) + NS * kTile * D * 2,
+                "candidates need the V ring and the extra slots to be adjacent");
+  static_assert(kCapH * 2 == kCap, "two equal halves");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;

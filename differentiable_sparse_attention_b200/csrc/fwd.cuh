@@ -285,6 +285,19 @@ __device__ __forceinline__ bool solver_step(double F0, double F1, double F2, flo
 constexpr int kFwdThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 
 __device__ __forceinline__ void fwd_epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// The same barrier, returning whether v held for any of the 256 threads.
+__device__ __forceinline__ bool fwd_epi_bar_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u)
+      : "memory");
+  return r != 0u;
+}
 
 // Per-row state that warpgroup 1 hands to warpgroup 0 at the end of a pass.
 struct FwdXrow {
@@ -328,6 +341,7 @@ struct FwdSmem {
   double xlo[kTile];          // 0 -> 1: bracket lower bound
   float xtau[kTile];          // 0 -> 1: current threshold
   int xflag[kTile];           // 0 -> 1: list rebuilt by COLLECT
+  int xact[kTile];            // 0 -> 1: the row still iterates over its lists
 };
 
 // Candidate scores live in the V ring and the slots after it, which stay idle
@@ -910,59 +924,71 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // ---------------- end of pass: merge the halves, solve, next tile list
       auto build_list = [&](double thr_d) {
         const float thr = row_ok ? __double2float_rd(thr_d) : INFINITY;
-        for (int t = 0; t < n; t += 4) {
-          float hv[4];
-          int jj[4];
+        // 16 tile maxima in flight per thread: the loads are latency-bound
+        constexpr int kU = 16;
+        for (int t = 0; t < n; t += kU) {
+          float hv[kU];
+          int jj[kU];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < kU; ++u) {
             jj[u] = (t + u < n) ? static_cast<int>(sm.tiles[t + u]) : -1;
             hv[u] = jj[u] >= 0 ? __half2float(P.tmax[tmax_index(bh, i, jj[u], P.tr, P.tc,
                                                                  P.causal) + wg * kTile + rl])
                                : -INFINITY;
           }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < kU; ++u) {
             const uint32_t b = __ballot_sync(0xffffffffu, hv[u] > thr);
             if (lane == 0 && b != 0u && jj[u] >= 0)
               atomicOr(&sm.flags[jj[u] >> 5], 1u << (jj[u] & 31));
           }
         }
       };
-      // Refinement over the row's candidate lists (warpgroup 0: both halves), in
-      // registers, once the lists hold every score above lo.
+      // Refinement over the row's candidate lists, in registers, once the lists
+      // hold every score above lo.  Each warpgroup sums over its own list;
+      // warpgroup 0 adds warpgroup 1's partial sums and takes the step.  All
+      // 256 epilogue threads run the same iterations (two barriers each) while
+      // any row of the tile still iterates.
       auto refine_registers = [&]() {
-        if (wg != 0 || !row_ok || cand_over || (collect && kind == PASS_HIST)) return;
-        // keep only the candidates above lo (the others contribute nothing at any
-        // tau >= lo), so the iterations run over roughly the support
-        {
-          const float thr = __double2float_rd(lo / P.c);
-          int kept = 0;
-          for (int a = 0; a < ncand; ++a) {
-            const float xa = my_cand[a * kTile];
-            if (xa > thr) my_cand[(kept++) * kTile] = xa;
-          }
-          ncand = kept;
-          kept = 0;
-          for (int a = 0; a < ncand1; ++a) {
-            const float xa = other_cand[a * kTile];
-            if (xa > thr) other_cand[(kept++) * kTile] = xa;
-          }
-          ncand1 = kept;
-          l_drop = fmax(l_drop, static_cast<double>(thr) * P.c);
+        bool act = false;
+        if (wg == 0) {
+          act = row_ok && !cand_over && !(collect && kind == PASS_HIST) && !row_done &&
+                iter < P.max_iter;
+          sm.xact[rl] = act ? 1 : 0;
+          sm.xtau[rl] = tau_c;
+          sm.xlo[rl] = lo;
         }
-        for (; iter < P.max_iter && !row_done;) {
+        bool first = true;
+        for (;;) {
+          if (!fwd_epi_bar_any(act)) break;
+          if (wg == 1) {
+            act = sm.xact[rl] != 0;
+            tau_c = sm.xtau[rl];
+          }
+          if (first && act) {
+            // keep only the candidates above lo (the others contribute nothing at
+            // any tau >= lo), so the iterations run over roughly the support
+            const double lo_r = wg == 0 ? lo : sm.xlo[rl];
+            const float thr = __double2float_rd(lo_r / P.c);
+            int kept = 0;
+            for (int a = 0; a < ncand; ++a) {
+              const float xa = my_cand[a * kTile];
+              if (xa > thr) my_cand[(kept++) * kTile] = xa;
+            }
+            ncand = kept;
+            if (wg == 0) l_drop = fmax(l_drop, static_cast<double>(thr) * P.c);
+          }
+          first = false;
           float f0[4] = {0.f, 0.f, 0.f, 0.f}, f1[4] = {0.f, 0.f, 0.f, 0.f},
                 f2[4] = {0.f, 0.f, 0.f, 0.f};
           float tmn[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
           float tng[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          const int ntot = ncand + ncand1;
-          for (int e0 = 0; e0 < ntot; e0 += 4) {
+          const int nown = act ? ncand : 0;
+          for (int e0 = 0; e0 < nown; e0 += 4) {
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
               const int e = e0 + a;
-              float tt = -INFINITY;
-              if (e < ncand) tt = fmaf(my_cand[e * kTile], P.c, -tau_c);
-              else if (e < ntot) tt = fmaf(other_cand[(e - ncand) * kTile], P.c, -tau_c);
+              const float tt = e < nown ? fmaf(my_cand[e * kTile], P.c, -tau_c) : -INFINITY;
               const bool in = tt > 0.0f;
               const float tp = fmaxf(tt, 0.0f);
               tmn[a] = in ? fminf(tmn[a], tt) : tmn[a];
@@ -983,15 +1009,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               }
             }
           }
-          const double F0c = (f0[0] + f0[1]) + (f0[2] + f0[3]);
-          const double F1c = (f1[0] + f1[1]) + (f1[2] + f1[3]);
-          const double F2c = (f2[0] + f2[1]) + (f2[2] + f2[3]);
-          const float tminc = fminf(fminf(tmn[0], tmn[1]), fminf(tmn[2], tmn[3]));
-          const float tnegc = fmaxf(fmaxf(tng[0], tng[1]), fmaxf(tng[2], tng[3]));
-          row_done = GEN ? solver_step_gen(F0c, F1c, F2c, P.kpow, tau_c, lo, hi, dx1, dx2)
-                         : solver_step<ALPHA2>(F0c, F1c, F2c, tminc, tnegc, l_drop, tau_c, lo, hi);
-          ++iter;
-          trace_store(iter, tau_c);
+          const float s0 = (f0[0] + f0[1]) + (f0[2] + f0[3]);
+          const float s1 = (f1[0] + f1[1]) + (f1[2] + f1[3]);
+          const float s2 = (f2[0] + f2[1]) + (f2[2] + f2[3]);
+          const float smin = fminf(fminf(tmn[0], tmn[1]), fminf(tmn[2], tmn[3]));
+          const float sneg = fmaxf(fmaxf(tng[0], tng[1]), fmaxf(tng[2], tng[3]));
+          if (wg == 1) {
+            sm.xf[0][rl] = s0;
+            sm.xf[1][rl] = s1;
+            sm.xf[2][rl] = s2;
+            sm.xtmin[rl] = smin;
+            sm.xtneg[rl] = sneg;
+          }
+          fwd_epi_bar();
+          if (wg == 0 && act) {
+            const double F0c = static_cast<double>(s0) + sm.xf[0][rl];
+            const double F1c = static_cast<double>(s1) + sm.xf[1][rl];
+            const double F2c = static_cast<double>(s2) + sm.xf[2][rl];
+            const float tminc = fminf(smin, sm.xtmin[rl]);
+            const float tnegc = fmaxf(sneg, sm.xtneg[rl]);
+            row_done = GEN ? solver_step_gen(F0c, F1c, F2c, P.kpow, tau_c, lo, hi, dx1, dx2)
+                           : solver_step<ALPHA2>(F0c, F1c, F2c, tminc, tnegc, l_drop, tau_c,
+                                                 lo, hi);
+            ++iter;
+            trace_store(iter, tau_c);
+            act = !row_done && iter < P.max_iter;
+            sm.xact[rl] = act ? 1 : 0;
+            sm.xtau[rl] = tau_c;
+          }
         }
       };
       // warpgroup 0 -> 1: the row's threshold, lower bound and COLLECT flag

@@ -323,8 +323,10 @@ struct FwdSmem {
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS];
   uint64_t v_full[NS], v_empty[NS];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2], o_full, drain;
+  // S buffers in TMEM: three at D = 64 (3 x 128 + 2 x 64 columns), two at 128
+  static constexpr int kNSB = D == 64 ? 3 : 2;
+  uint64_t s_full[kNSB], s_empty[kNSB];
+  uint64_t p_full[kNSB], p_empty[kNSB], o_full, drain;
   uint32_t tmem_base;
   int abort_flag;
   int ctl_kind, ctl_n, ctl_iter;
@@ -394,8 +396,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t idesc_pv = P.vbar != nullptr ? make_idesc(kTile, D, 0, 0, 0, 1)
                                               : make_idesc(kTile, D, 1, 1, 0, 1);
   const bool gv = P.vbar != nullptr;
-  constexpr uint32_t kColO = 256;      // TMEM: S0, S1 (P / G of the P.V pass), O, G.V
-  constexpr uint32_t kColG = 256 + D;
+  constexpr uint32_t kNSB = Smem::kNSB;
+  constexpr uint32_t kColO = kNSB * kTile;   // TMEM: S buffers (P / G of the P.V pass), O, G.V
+  constexpr uint32_t kColG = kColO + D;
+  static_assert(kColG + D <= 512, "TMEM columns");
   constexpr int kCap = fwd_cand_cap<D, NS>();
   constexpr int kCapH = kCap / 2;
   static_assert(offsetof(Smem, cx) == offsetof(Smem, v) + NS * kTile * D * 2,
@@ -417,11 +421,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < static_cast<int>(kNSB); ++s) {
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.s_empty[s], 8);
-    }
-    for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.p_full[s], 8);
       mbar_init(&sm.p_empty[s], 1);
     }
@@ -574,7 +576,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         auto issue_s = [&]() -> bool {
           const uint32_t slot = kc % NS;
           if (!mbar_wait(&sm.k_full[slot], (kc / NS) & 1, abort_flag, P.status)) return false;
-          const uint32_t sb = sc & 1, use = sc >> 1;
+          const uint32_t sb = sc % kNSB, use = sc / kNSB;
           if (use > 0 && !mbar_wait(&sm.s_empty[sb], (use - 1) & 1, abort_flag, P.status))
             return false;
           tc_fence_after();
@@ -595,12 +597,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // P and G sit in the S buffer of their tile: 32-key chunk c occupies
         // columns 32 c .. 32 c + 31, P packed in the first 16, G in the last 16.
         auto issue_pv = [&](uint32_t sc0) -> bool {
-          const uint32_t pb = pc & 1;
-          if (!mbar_wait(&sm.p_full[pb], (pc >> 1) & 1, abort_flag, P.status)) return false;
+          const uint32_t pb = pc % kNSB;
+          if (!mbar_wait(&sm.p_full[pb], (pc / kNSB) & 1, abort_flag, P.status)) return false;
           const uint32_t slot = vc % NS;
           if (!mbar_wait(&sm.v_full[slot], (vc / NS) & 1, abort_flag, P.status)) return false;
           tc_fence_after();
-          const uint32_t t_p = tmem + ((sc0 + pc) & 1) * kTile;
+          const uint32_t t_p = tmem + ((sc0 + pc) % kNSB) * kTile;
           const uint32_t v_addr = smem_u32(sm.v[slot]);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk) {
@@ -622,9 +624,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           } else {
             const uint32_t sc0 = sc;
             for (int t = 0; t <= n && ok; ++t) {
-              // S(t) reuses the TMEM buffer of P.V tile t - 2: wait for its MMAs
-              if (t < n && t >= 2)
-                ok = mbar_wait(&sm.p_empty[t & 1], ((t - 2) >> 1) & 1, abort_flag, P.status);
+              // S(t) reuses the TMEM buffer of P.V tile t - kNSB: wait for its MMAs
+              if (t < n && t >= static_cast<int>(kNSB))
+                ok = mbar_wait(&sm.p_empty[t % kNSB], ((t / kNSB) - 1) & 1, abort_flag,
+                               P.status);
               if (ok && t < n) ok = issue_s();
               if (ok && t > 0) ok = issue_pv(sc0);
             }
@@ -646,8 +649,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int t = 0; t < n; ++t) {
         const int j = sm.tiles[t];
         const uint32_t cur = sc++;
-        const uint32_t sb = cur & 1;
-        ok = mbar_wait(&sm.s_full[sb], (cur >> 1) & 1, abort_flag, P.status);
+        const uint32_t sb = cur % kNSB;
+        ok = mbar_wait(&sm.s_full[sb], (cur / kNSB) & 1, abort_flag, P.status);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
@@ -850,7 +853,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         } else {  // PASS_PV
           // P (and G) replace the scores in this S buffer; the MMA warp issues
           // S(t + 2) into it only after the P.V MMAs of this tile completed.
-          const uint32_t pb = pc & 1;
+          const uint32_t pb = pc % kNSB;
           ++pc;
           float part = 0.f, gpart = 0.f;
 #pragma unroll 1

@@ -27,7 +27,7 @@ DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
 EXPORTED = ("entmax_attn_mask_words", "entmax_attn_workspace_size", "entmax_attn_fwd",
             "entmax_attn_bwd", "entmax_attn_status", "entmax_attn_counters",
             "entmax_attn_profile", "entmax_attn_profile_read", "entmax_attn_error_string",
-            "entmax_attn_fwd_noalloc")
+            "entmax_attn_fwd_noalloc", "entmax_attn_wait_selftest")
 # include/dash_route.h: the DashAttention stage-0/1 router
 DASH_EXPORTED = ("dash_route_workspace_size", "dash_route_fwd")
 DASH_MAX_CHUNKS = 256
@@ -78,6 +78,8 @@ def _lib():
     lib.entmax_attn_fwd_noalloc.restype = c_int
     lib.entmax_attn_error_string.argtypes = [c_int]
     lib.entmax_attn_error_string.restype = ctypes.c_char_p
+    lib.entmax_attn_wait_selftest.argtypes = [vp, vp, ctypes.c_ulonglong, vp]
+    lib.entmax_attn_wait_selftest.restype = c_int
     lib.dash_route_workspace_size.argtypes = [c_int] * 6
     lib.dash_route_workspace_size.restype = c_size
     lib.dash_route_fwd.argtypes = ([vp, vp] + [c_int] * 6 + [c_float, c_float, c_int]

@@ -17,6 +17,8 @@
 //                           query tiles, accumulated in TMEM (no atomics).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace entmax {
@@ -391,21 +393,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const int col0 = j * kTile + wg * kHalf;
       const bool msk = (P.causal && j == i) || (col0 + kHalf > P.N);
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t rs[32], rp[32];
-        tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
-        uint32_t w[16];
+      // dS of one 32-key chunk; MASKED (diagonal and tail tiles only) drops the
+      // keys at or beyond `nv` -- a tile-uniform choice, so the common path
+      // carries no per-key test
+      auto chunk_ds = [&](auto masked_tag, const int ch, const uint32_t (&rs)[32],
+                          const uint32_t (&rp)[32], uint32_t (&w)[16]) {
+        constexpr bool MASKED = decltype(masked_tag)::value;
+        int nv = 32;
+        if constexpr (MASKED)
+          nv = min(32, max(0, (P.causal ? min(row + 1, P.N) : P.N) - (col0 + ch * 32)));
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           float g2[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             float tt = fmaf(__uint_as_float(rs[2 * e + u]), P.c, -tau_r);
-            if (msk) {
-              const int col = col0 + ch * 32 + 2 * e + u;
-              if (!(col < P.N && (!P.causal || col <= row))) tt = -1.0f;
-            }
+            if constexpr (MASKED) tt = (2 * e + u < nv) ? tt : -1.0f;
             if (GEN)   // g = t^(k - 1) <= 1 (alpha <= 2: k >= 1, t <= 1)
               g2[u] = tt > 0.f ? __fdividef(pow_pos(tt, P.kpow), tt) : 0.f;
             else
@@ -416,6 +419,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const __half2 h2 = __floats2half2_rn(d0, d1);
           w[e] = *reinterpret_cast<const uint32_t*>(&h2);
         }
+      };
+#pragma unroll 1
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t rs[32], rp[32];
+        tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
+        uint32_t w[16];
+        if (msk) chunk_ds(std::true_type{}, ch, rs, rp, w);
+        else chunk_ds(std::false_type{}, ch, rs, rp, w);
         tmem_st16(t_s + ch * 32, w);   // dS over the S chunk just read
       }
       tmem_wait_st();
@@ -679,11 +690,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const int row0 = it * kTile + wg * kHalf;
       const bool msk = (P.causal && it == j) || (row0 + kHalf > P.N) || !key_ok;
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t rs[32], rp[32];
-        tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
-        uint32_t wp[16], wd[16];
+      // P^T and dS^T of one 32-row chunk; MASKED (diagonal and tail tiles only)
+      // keeps rows in [lo_v, hi_v) of the chunk -- a tile-uniform choice
+      auto chunk_pds = [&](auto masked_tag, const int ch, const uint32_t (&rs)[32],
+                           const uint32_t (&rp)[32], uint32_t (&wp)[16], uint32_t (&wd)[16]) {
+        constexpr bool MASKED = decltype(masked_tag)::value;
+        int lo_v = 0, hi_v = 32;
+        if constexpr (MASKED) {
+          const int r0 = row0 + ch * 32;
+          lo_v = P.causal ? max(0, key - r0) : 0;
+          hi_v = key_ok ? min(32, max(0, P.N - r0)) : 0;
+        }
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const int r4 = wg * kHalf + ch * 32 + e;
@@ -695,11 +712,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             float tt = fmaf(__uint_as_float(rs[e + u]), P.c, -taus[u]);
-            if (msk) {
-              const int row = row0 + ch * 32 + e + u;
-              const bool ok_e = key_ok && row < P.N && (!P.causal || key <= row);
-              if (!ok_e) tt = -1.0f;
-            }
+            if constexpr (MASKED) tt = (e + u >= lo_v && e + u < hi_v) ? tt : -1.0f;
             const float tp = fmaxf(tt, 0.0f);
             float g;
             if (GEN) {
@@ -720,6 +733,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           wd[e / 2] = *reinterpret_cast<uint32_t*>(&b0);
           wd[e / 2 + 1] = *reinterpret_cast<uint32_t*>(&b1);
         }
+      };
+#pragma unroll 1
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t rs[32], rp[32];
+        tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
+        uint32_t wp[16], wd[16];
+        if (msk) chunk_pds(std::true_type{}, ch, rs, rp, wp, wd);
+        else chunk_pds(std::false_type{}, ch, rs, rp, wp, wd);
         tmem_st16(t_s + ch * 32, wp);    // P^T over the S^T chunk just read
         tmem_st16(t_dp + ch * 32, wd);   // dS^T over the dP^T chunk
       }

@@ -31,6 +31,27 @@ __device__ __forceinline__ float pow_pos(float t, float e) {
   return t > 0.0f ? exp2f(e * __log2f(t)) : 0.0f;
 }
 
+// Exercises the bounded wait: one thread waits on an mbarrier that no thread
+// arrives at, with a limit of limit_ns.  The wait gives up, raises the abort
+// flag and ST_TIMEOUT in *status exactly as in the attention kernels, and the
+// kernel returns; result[0] = 1 once it has returned from the wait.
+__global__ void wait_selftest_kernel(uint32_t* status, uint32_t* result, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+    result[0] = 1u;
+    result[1] = ok ? 1u : 0u;
+    result[2] = abort_flag ? 1u : 0u;
+  }
+}
+
 enum PassKind : int { PASS_HIST = 0, PASS_REFINE = 1, PASS_PV = 2, PASS_DONE = 3, PASS_COLLECT = 4 };
 
 // Work counters kept in the workspace right after the status word (uint64 each).

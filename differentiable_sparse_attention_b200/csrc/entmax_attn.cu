@@ -703,6 +703,20 @@ int dash_route_fwd(const void* q, const void* k, int B, int Hq, int Hkv, int N, 
   }
 }
 
+int entmax_attn_wait_selftest(void* workspace, uint32_t* result, unsigned long long limit_ns,
+                              void* stream) {
+  if (!workspace || !result) return ENTMAX_E_NULL;
+  if (limit_ns < 1 || limit_ns > 1000000000ull) return ENTMAX_E_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      (reinterpret_cast<uintptr_t>(result) & 3u) != 0)
+    return ENTMAX_E_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return ENTMAX_E_CUDA;
+  if (cudaMemsetAsync(result, 0, 3 * sizeof(uint32_t), st) != cudaSuccess) return ENTMAX_E_CUDA;
+  wait_selftest_kernel<<<1, 32, 0, st>>>(static_cast<uint32_t*>(workspace), result, limit_ns);
+  return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
+}
+
 const char* entmax_attn_error_string(int code) {
   switch (code) {
     case ENTMAX_OK: return "success";

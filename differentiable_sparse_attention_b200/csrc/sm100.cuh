@@ -79,13 +79,13 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kWaitSleepNs = 20000u;   // suspend-time hint per try_wait
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
+                                          uint32_t* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if (abort_flag != nullptr && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       if (abort_flag != nullptr) *abort_flag = 1;
       if (status != nullptr) atomicOr(status, ST_TIMEOUT);
       return false;

@@ -207,6 +207,18 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Diagnostics of the failure handling (the pages have no counterpart): runs a
+ * one-thread kernel that waits on an mbarrier nothing ever arrives at, with a
+ * limit of limit_ns nanoseconds (1..10^9) instead of the kernels' 2 s, so the
+ * bounded wait runs out: it raises ENTMAX_ST_TIMEOUT in `workspace`'s status
+ * word (cleared first) and the kernel returns.  result: device uint32[3],
+ * written [1 = returned, 1 = the wait succeeded, 1 = abort flag raised].  No
+ * fault, trap or unbounded loop is involved; the context stays usable.
+ */
+int entmax_attn_wait_selftest(void* workspace, uint32_t* result, unsigned long long limit_ns,
+                              void* stream);
+
+/*
  * Synchronises `stream` and copies the device status word (ENTMAX_ST_* bits)
  * of `workspace` to *status.  Returns ENTMAX_E_CUDA if the stream reported an
  * error (e.g. from an earlier launch).

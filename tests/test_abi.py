@@ -111,3 +111,11 @@ def test_error_strings(lib):
     for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -99):
         s = dsa.error_string(code)
         assert isinstance(s, str) and s
+
+
+def test_wait_selftest_validation(lib):
+    assert lib.entmax_attn_wait_selftest(None, FAKE, 1000, None) == dsa.E_NULL
+    assert lib.entmax_attn_wait_selftest(FAKE, None, 1000, None) == dsa.E_NULL
+    assert lib.entmax_attn_wait_selftest(FAKE, FAKE, 0, None) == dsa.E_SHAPE
+    assert lib.entmax_attn_wait_selftest(FAKE, FAKE, 2_000_000_000, None) == dsa.E_SHAPE
+    assert lib.entmax_attn_wait_selftest(MISALIGNED, FAKE, 1000, None) == dsa.E_ALIGN

@@ -30,6 +30,8 @@
 
 #include <cstddef>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace entmax {
@@ -865,6 +867,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (msk) apply_mask(v, j, ch);
             uint32_t w[16], wgt[16];
+            // p (and g) of the chunk packed for the tensor core: fp16 P and G with
+            // the g-weighted means, bf16 P without -- a per-launch choice, so the
+            // score loop is instantiated for each
+            auto pv_chunk = [&](auto gv_tag) {
+            constexpr bool GV = decltype(gv_tag)::value;
             float ps[4] = {0.f, 0.f, 0.f, 0.f}, gs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -886,8 +893,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 g1 = ALPHA2 ? (t1 > 0.0f ? 1.0f : 0.0f) : t1;
               }
               ps[e & 3] += p0 + p1;
-              gs[e & 3] += g0 + g1;
-              if (gv) {
+              if constexpr (GV) {
+                gs[e & 3] += g0 + g1;
                 const __half2 h2 = __floats2half2_rn(p0, p1);
                 const __half2 g2 = __floats2half2_rn(g0, g1);
                 w[e] = *reinterpret_cast<const uint32_t*>(&h2);
@@ -899,6 +906,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             part += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             gpart += (gs[0] + gs[1]) + (gs[2] + gs[3]);
+            };
+            if (gv) pv_chunk(std::true_type{});
+            else pv_chunk(std::false_type{});
             tmem_st16(t_s + ch * 32, w);
             if (gv) tmem_st16(t_s + ch * 32 + 16, wgt);
           }

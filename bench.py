@@ -67,6 +67,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "sm_max_mhz": 1965.0}
 
 
+# Algorithmic ALU work per score of the forward's passes (lane-ops): running max
+# and binning in the histogram pass, the sums of a refinement pass, t, p and the
+# packing of the P.V pass.
+ALU_OPS_HIST, ALU_OPS_REFINE, ALU_OPS_PV = 8, 6, 3
+
+
 def max_over_ranks(x: float, device=None) -> float:
     """The maximum of x over the ranks of the default process group (x itself
     without one); the tensor lives on `device` (a CUDA device under NCCL)."""
@@ -309,6 +315,28 @@ def run_ours(args, points, rank, world, device):
         roof["traffic"] = tr["bytes"]
         roof["traffic_from"] = tr["from"]
 
+    # the forward's tau passes are bound by the plain ALU pipes, not the tensor
+    # cores: the same kernel against 128 lanes x 148 SMs x the clock
+    roof_alu = None
+    if "fwd" in phase_tot:
+        fwd_ms = phase_tot["fwd"] / n_steps_all
+        ops = 0.0
+        for w, r in zip(points, results):
+            c = r["counters"]
+            scores = 128.0 * 128.0
+            ops += (ALU_OPS_HIST * c["fwd_hist_tiles"] + ALU_OPS_REFINE * c["fwd_refine_tiles"]
+                    + ALU_OPS_PV * c["fwd_pv_tiles"]) * scores
+        ops /= len(points)
+        sm_mhz = peaks.get("sm_max_mhz", 1965.0)
+        alu_peak = 128 * 148 * sm_mhz * 1e6 / 1e12     # T lane-ops/s
+        achieved = ops / (fwd_ms * 1e-3) / 1e12
+        roof_alu = {"bound": "alu", "kernel": "fwd", "achieved": round(achieved, 3),
+                    "peak": round(alu_peak, 2), "unit": "T lane-ops/s",
+                    "frac": round(achieved / alu_peak, 4),
+                    "note": f"{ALU_OPS_HIST} ops per histogram score, {ALU_OPS_REFINE} per "
+                            f"refinement score, {ALU_OPS_PV} per P.V score over the tiles the "
+                            f"counters report; peak = 128 lanes x 148 SMs x {sm_mhz:g} MHz"}
+
     line = {
         "metric": "fwd+bwd alpha-entmax attn ms/step & effective TFLOP/s vs block sparsity, 1 B200",
         "value": round(value, 3),
@@ -322,6 +350,7 @@ def run_ours(args, points, rank, world, device):
         "sweep": results,
         "kernels_ms_per_step": {n: round(v / n_steps_all, 4) for n, v in phase_tot.items()},
         "roofline": roof,
+        "roofline_fwd_alu": roof_alu,
         "gpu_launches": kernel_launches,
         "clocks": merge_clocks([r["clocks"] for r in results]),
     }

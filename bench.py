@@ -43,11 +43,11 @@ from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
 # and kernel, valid only for the kernel sources they were taken on (hash of
 # the package's csrc/); any other source reports traffic as null.
 TRAFFIC = {
-    ("alpha15_4k", "fwd"): {"bytes": 67736064, "src": "7fd941a9c33ccf58",
+    ("alpha15_4k", "fwd"): {"bytes": 67979264, "src": "ed116934f7f065d6",
                             "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_row"): {"bytes": 109964288, "src": "7fd941a9c33ccf58",
+    ("alpha15_4k", "bwd_row"): {"bytes": 109290752, "src": "ed116934f7f065d6",
                                 "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_col"): {"bytes": 75369472, "src": "7fd941a9c33ccf58",
+    ("alpha15_4k", "bwd_col"): {"bytes": 75350784, "src": "ed116934f7f065d6",
                                 "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
 }
 

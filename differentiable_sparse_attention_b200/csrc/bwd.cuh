@@ -152,7 +152,6 @@ __device__ __forceinline__ int load_tile_list(const uint32_t* rowbits, int wt, u
 // Two epilogue warpgroups (warps 2-5 and 6-9) alternate: warpgroup h owns half
 // h of every tile and its TMEM / SMEM buffer.
 constexpr int kBwdThreads = 320;
-constexpr int kBwdEpi = 256;
 constexpr int kHalf = 64;
 constexpr int kHalfBytes = kTile * kHalf * 2;   // one [128][64] fp16 slab
 

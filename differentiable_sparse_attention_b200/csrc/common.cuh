@@ -11,8 +11,6 @@
 namespace entmax {
 
 constexpr int kTile = 128;                   // compute tile: 128 query rows x 128 keys
-constexpr int kThreads = 192;                // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kEpiThreads = 128;
 constexpr int kMaxN = 262144;
 constexpr int kMaxTiles = kMaxN / kTile;     // 2048 tiles per row
 constexpr int kMaxMaskWords = kMaxN / 64 / 32;  // words per mask row at block 64
@@ -67,9 +65,6 @@ enum Counter : int {
 };
 
 
-// Named barrier over the four epilogue warps only (id 1; id 0 is __syncthreads).
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
 // 64-bit left shift with the PTX clamp rule: a shift amount >= 64 (including
 // "negative" amounts seen as huge unsigned values) yields 0.
 __device__ __forceinline__ uint64_t shl64(uint64_t x, uint32_t sh) {
@@ -87,16 +82,6 @@ __device__ __forceinline__ size_t tmax_index(int bh, int i, int j, int tr, int t
   const size_t idx = causal ? static_cast<size_t>(i) * (i + 1) / 2 + j
                             : static_cast<size_t>(i) * tc + j;
   return (static_cast<size_t>(bh) * per + idx) * (2 * kTile);
-}
-
-// Byte offset, inside a 128-byte-swizzled K-major tile made of [128 rows][64
-// bf16] slabs, of the 16-byte chunk holding elements [8c, 8c+8) of row `row`
-// (element index counted across slabs).  The tensor core and TMA apply the
-// same XOR of address bits [4,7) with bits [7,10).
-__device__ __forceinline__ uint32_t sw128_chunk_offset(int row, int chunk16) {
-  const int slab = chunk16 >> 3;
-  const int c = chunk16 & 7;
-  return static_cast<uint32_t>(slab * kSlabBytes + row * 128 + ((c ^ (row & 7)) << 4));
 }
 
 // Maximum of 32 values as a 5-level tree (a linear chain would serialise 31

@@ -43,11 +43,11 @@ from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
 # and kernel, valid only for the kernel sources they were taken on (hash of
 # the package's csrc/); any other source reports traffic as null.
 TRAFFIC = {
-    ("alpha15_4k", "fwd"): {"bytes": 67979264, "src": "ed116934f7f065d6",
+    ("alpha15_4k", "fwd"): {"bytes": 67928576, "src": "31411802dc754e86",
                             "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_row"): {"bytes": 109290752, "src": "ed116934f7f065d6",
+    ("alpha15_4k", "bwd_row"): {"bytes": 109537792, "src": "31411802dc754e86",
                                 "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_col"): {"bytes": 75350784, "src": "ed116934f7f065d6",
+    ("alpha15_4k", "bwd_col"): {"bytes": 77797120, "src": "31411802dc754e86",
                                 "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
 }
 

@@ -40,16 +40,25 @@ sys.path.insert(0, ROOT)
 from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
 
 # DRAM bytes (read + write) per launch from one ncu capture, keyed by workload
-# and kernel, valid only for the kernel sources they were taken on (hash of
-# the package's csrc/); any other source reports traffic as null.
+# and kernel, valid only for the kernel code they were taken on (hash of the
+# package's csrc/ with comments and white space removed); any other code
+# reports traffic as null.
 TRAFFIC = {
-    ("alpha15_4k", "fwd"): {"bytes": 67928576, "src": "31411802dc754e86",
+    ("alpha15_4k", "fwd"): {"bytes": 67928576, "src": "78caf74992c7b235",
                             "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_row"): {"bytes": 109537792, "src": "31411802dc754e86",
+    ("alpha15_4k", "bwd_row"): {"bytes": 109537792, "src": "78caf74992c7b235",
                                 "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_col"): {"bytes": 77797120, "src": "31411802dc754e86",
+    ("alpha15_4k", "bwd_col"): {"bytes": 77797120, "src": "78caf74992c7b235",
                                 "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
 }
+
+
+def _code_only(text: str) -> str:
+    """C++ source without comments and blank space: what the compiler sees."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
 
 
 def kernel_source_hash() -> str:
@@ -58,8 +67,8 @@ def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "differentiable_sparse_attention_b200", "csrc", "*"))):
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -17,15 +17,18 @@
 //           tau* - h <= tau_h <= tau* (Proposition 1, as the summaries state it),
 //           and the safeguarded Halley (alpha = 1.5) / Newton (alpha = 2) steps
 //           (zh §2.2, it §2B, ja §2.2, es §2B) then run in registers over the
-//           candidates until the threshold is certified exact.
+//           candidates until the threshold is certified exact (other alpha:
+//           powers t^k and a tolerance instead of the certificate).
 //   COLLECT (only if a candidate list overflowed) rebuilds the lists above the
 //           final lower bound.
 //   REFINE  (only if a rebuilt list still overflows) refinement steps that
 //           stream the key tiles again.
 //   PV      tiles whose recorded maximum exceeds the row's lower bound:
-//           p = [s - tau]_+^(1/(alpha-1)) written to SMEM as bf16, O += P V on the
-//           tensor cores, and the bit-packed block mask (32 blocks per uint32
-//           word, zh §2.3) of blocks holding a p > 0.
+//           p = [s - tau]_+^(1/(alpha-1)) and g = p^(2-alpha) written as fp16 over
+//           the scores in TMEM, O += P V and G.V += G V on the tensor cores (A
+//           read from TMEM, V an fp16 copy), the bit-packed block mask (32 blocks
+//           per uint32 word, zh §2.3) of blocks holding a p > 0, and per row the
+//           g-weighted mean of v, G.V / sum g, which the backward's delta needs.
 #pragma once
 
 #include <cstddef>
@@ -1069,8 +1072,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // Publish the next pass: PV unless some row still needs its list rebuilt
       // (COLLECT) or must refine over the key tiles (REFINE).
       auto next_pass = [&](int passes_done_kind) {
-        // the candidate slots are V-ring / P-tile memory that TMA and the
-        // tensor core use next: order these generic accesses before them
+        // the candidate slots are V-ring memory that TMA and the tensor core
+        // use next: order these generic accesses before them
         fence_proxy_async_smem();
         build_list(lo);
         fwd_epi_bar();

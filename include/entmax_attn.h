@@ -153,10 +153,13 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
  * allocator).  The paper has no counterpart to this entry point; it exists
  * only for such callers.
  *
- * It computes exactly what entmax_attn_fwd computes (same kernel, same
- * arguments and outputs, no tau_trace), but its scratch -- status word, work
- * counters and the histogram pass's tile maxima -- lives in one fixed device
- * array of ENTMAX_NOALLOC_SCRATCH_BYTES (8 MiB) that is part of this library:
+ * It runs the kernel of entmax_attn_fwd with the same arguments and outputs
+ * (no tau_trace): tau and the mask are the same, and O differs only in the
+ * rounding of P, which is bf16 here (it multiplies v itself, as no fp16 copy
+ * of v fits the scratch) instead of fp16.  It forms no g-weighted means, so
+ * entmax_attn_bwd cannot follow it.  Its scratch -- status word, work counters
+ * and the histogram pass's tile maxima -- lives in one fixed device array of
+ * ENTMAX_NOALLOC_SCRATCH_BYTES (8 MiB) that is part of this library:
  * every GPU that loads the library holds those 8 MiB until the process exits.
  * The call allocates nothing and calls no allocating routine.
  *   - Problems whose scratch exceeds the 8 MiB return ENTMAX_E_SCRATCH and

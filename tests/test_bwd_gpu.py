@@ -4,7 +4,8 @@ float64 oracle's gradients through the entmax Jacobian."""
 import pytest
 import torch
 
-from differentiable_sparse_attention_b200 import entmax_attn_bwd, entmax_attn_fwd, status
+from differentiable_sparse_attention_b200 import (entmax_attention, entmax_attn_bwd, entmax_attn_fwd,
+                                                status)
 from differentiable_sparse_attention_b200.workloads import Workload, make_inputs
 from parity import check_grads_head, to64
 
@@ -49,3 +50,19 @@ def test_backward_deterministic(cuda_device):
                         workspace=f.workspace)
     for ga, gb in zip(a, b):
         assert torch.equal(ga, gb)
+
+
+def test_autograd_wrapper_matches_the_explicit_calls(cuda_device):
+    # entmax_attention through torch.autograd gives the same gradients, bit for
+    # bit, as entmax_attn_fwd followed by entmax_attn_bwd on the same inputs
+    w = Workload("autograd", B=1, H=2, N=300, D=64, alpha=1.5, temperature=2.0, seed=9)
+    x = make_inputs(w, device=cuda_device)
+    q, k, v = (x[n].detach().clone().requires_grad_(True) for n in ("q", "k", "v"))
+    o = entmax_attention(q, k, v, 1.5, True, 128)
+    o.backward(x["dout"])
+    f = entmax_attn_fwd(x["q"], x["k"], x["v"], 1.5, True, 128)
+    dq, dk, dv = entmax_attn_bwd(x["q"], x["k"], x["v"], x["dout"], f.tau, f.mask, 1.5, True,
+                                 128, workspace=f.workspace)
+    assert torch.equal(o.detach(), f.out)
+    for got, want in ((q.grad, dq), (k.grad, dk), (v.grad, dv)):
+        assert torch.equal(got, want)

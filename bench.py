@@ -44,12 +44,12 @@ from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
 # package's csrc/ with comments and white space removed); any other code
 # reports traffic as null.
 TRAFFIC = {
-    ("alpha15_4k", "fwd"): {"bytes": 67928576, "src": "78caf74992c7b235",
-                            "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_row"): {"bytes": 109537792, "src": "78caf74992c7b235",
-                                "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_col"): {"bytes": 77797120, "src": "78caf74992c7b235",
-                                "from": "profiles/full_alpha15_n4096_d64_t1.md (t = 1 launch)"},
+    ("alpha15_4k", "fwd"): {"bytes": 67279872, "src": "d4da4de491e110e1",
+                            "from": "profiles/dram_alpha15_n4096_d64_t1.md (t = 1 launch)"},
+    ("alpha15_4k", "bwd_row"): {"bytes": 105892608, "src": "d4da4de491e110e1",
+                                "from": "profiles/dram_alpha15_n4096_d64_t1.md (t = 1 launch)"},
+    ("alpha15_4k", "bwd_col"): {"bytes": 72186880, "src": "d4da4de491e110e1",
+                                "from": "profiles/dram_alpha15_n4096_d64_t1.md (t = 1 launch)"},
 }
 
 

@@ -65,6 +65,13 @@ enum Counter : int {
 };
 
 
+// a * b + c clamped to [0, 1] in one instruction (a NaN result becomes 0).
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 64-bit left shift with the PTX clamp rule: a shift amount >= 64 (including
 // "negative" amounts seen as huge unsigned values) yields 0.
 __device__ __forceinline__ uint64_t shl64(uint64_t x, uint32_t sh) {

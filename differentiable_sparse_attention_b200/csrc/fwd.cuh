@@ -876,37 +876,64 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             auto pv_chunk = [&](auto gv_tag) {
             constexpr bool GV = decltype(gv_tag)::value;
             float ps[4] = {0.f, 0.f, 0.f, 0.f}, gs[4] = {0.f, 0.f, 0.f, 0.f};
+            __half2 gcount = __float2half2_rn(0.0f);   // alpha = 2: support size
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float t0 = fmaxf(fmaf(v[2 * e], P.c, -tau_c), 0.0f);
-              const float t1 = fmaxf(fmaf(v[2 * e + 1], P.c, -tau_c), 0.0f);
-              float p0, p1, g0, g1;
               if (GEN) {
+                const float t0 = fmaxf(fmaf(v[2 * e], P.c, -tau_c), 0.0f);
+                const float t1 = fmaxf(fmaf(v[2 * e + 1], P.c, -tau_c), 0.0f);
                 // g = t^(k - 1), held below 6e4 (fp16) where alpha > 2 lets it grow
                 // without bound at the edge of the support
-                p0 = pow_pos(t0, P.kpow);
-                p1 = pow_pos(t1, P.kpow);
-                g0 = t0 > 0.0f ? fminf(__fdividef(p0, t0), 6.0e4f) : 0.0f;
-                g1 = t1 > 0.0f ? fminf(__fdividef(p1, t1), 6.0e4f) : 0.0f;
+                const float p0 = pow_pos(t0, P.kpow);
+                const float p1 = pow_pos(t1, P.kpow);
+                const float g0 = t0 > 0.0f ? fminf(__fdividef(p0, t0), 6.0e4f) : 0.0f;
+                const float g1 = t1 > 0.0f ? fminf(__fdividef(p1, t1), 6.0e4f) : 0.0f;
+                ps[e & 3] += p0 + p1;
+                if constexpr (GV) {
+                  gs[e & 3] += g0 + g1;
+                  const __half2 h2 = __floats2half2_rn(p0, p1);
+                  const __half2 g2 = __floats2half2_rn(g0, g1);
+                  w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                  wgt[e] = *reinterpret_cast<const uint32_t*>(&g2);
+                } else {
+                  const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                  w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
               } else {
-                p0 = ALPHA2 ? t0 : t0 * t0;
-                p1 = ALPHA2 ? t1 : t1 * t1;
-                // g = p^(2 - alpha): the support indicator at alpha = 2, t at 1.5
-                g0 = ALPHA2 ? (t0 > 0.0f ? 1.0f : 0.0f) : t0;
-                g1 = ALPHA2 ? (t1 > 0.0f ? 1.0f : 0.0f) : t1;
-              }
-              ps[e & 3] += p0 + p1;
-              if constexpr (GV) {
-                gs[e & 3] += g0 + g1;
-                const __half2 h2 = __floats2half2_rn(p0, p1);
-                const __half2 g2 = __floats2half2_rn(g0, g1);
-                w[e] = *reinterpret_cast<const uint32_t*>(&h2);
-                wgt[e] = *reinterpret_cast<const uint32_t*>(&g2);
-              } else {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                // p = t^k <= 1 with sum p = 1, so t lies in [0, 1] at tau*: the
+                // clamp to the support is a saturating FMA
+                const float t0 = fma_sat(v[2 * e], P.c, -tau_c);
+                const float t1 = fma_sat(v[2 * e + 1], P.c, -tau_c);
+                if constexpr (GV) {
+                  const __half2 th = __floats2half2_rn(t0, t1);
+                  if (ALPHA2) {
+                    // p = t; g = 1 on the support, counted exactly in half2
+                    const __half2 g2 = __hgt2(th, __float2half2_rn(0.0f));
+                    gcount = __hadd2(gcount, g2);
+                    ps[(2 * e) & 3] += t0;
+                    ps[(2 * e + 1) & 3] += t1;
+                    w[e] = *reinterpret_cast<const uint32_t*>(&th);
+                    wgt[e] = *reinterpret_cast<const uint32_t*>(&g2);
+                  } else {
+                    // g = t, and p = t^2 squared from the fp16 t
+                    const __half2 p2 = __hmul2(th, th);
+                    ps[(2 * e) & 3] = fmaf(t0, t0, ps[(2 * e) & 3]);
+                    ps[(2 * e + 1) & 3] = fmaf(t1, t1, ps[(2 * e + 1) & 3]);
+                    gs[(2 * e) & 3] += t0;
+                    gs[(2 * e + 1) & 3] += t1;
+                    w[e] = *reinterpret_cast<const uint32_t*>(&p2);
+                    wgt[e] = *reinterpret_cast<const uint32_t*>(&th);
+                  }
+                } else {
+                  const float p0 = ALPHA2 ? t0 : t0 * t0;
+                  const float p1 = ALPHA2 ? t1 : t1 * t1;
+                  ps[e & 3] += p0 + p1;
+                  const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                  w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
               }
             }
+            if (ALPHA2 && GV) gs[0] = __low2float(gcount) + __high2float(gcount);
             part += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             gpart += (gs[0] + gs[1]) + (gs[2] + gs[3]);
             };

@@ -1,0 +1,122 @@
+"""bench.py's host-side arithmetic and the reference arm's JSON line, on CPU.
+
+These cover what the numbers in bench.py's line are made of:
+- the dense-equivalent FLOP convention;
+- block sparsity read from the bit-packed mask;
+- the MMA FLOPs that the tile counters imply for each kernel's roofline;
+- the comment-insensitive hash that keys the measured DRAM traffic;
+- the fields of the reference arm (the oracle on the host cores).
+"""
+
+import os
+import sys
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
+
+
+def test_effective_flops_convention():
+    # forward 4 N^2 D per head (halved when causal), backward 2.5 x the forward
+    w = W.ALPHA15_4K
+    assert bench.effective_flops(w) == 7.0 * 2 * 16 * 4096 * 4096 * 64
+    assert bench.effective_flops(w.with_(causal=False)) == 2 * bench.effective_flops(w)
+
+
+def _mask(B, H, tb, rows):
+    """int32 mask words [B, H, tb, ceil(tb / 32)] with the given (i, j) bits set
+    in every head."""
+    words = (tb + 31) // 32
+    m = torch.zeros((B, H, tb, words), dtype=torch.int64)
+    for i, j in rows:
+        m[..., i, j // 32] |= 1 << (j % 32)
+    # the library stores uint32 bit patterns in int32 tensors
+    return torch.where(m >= 2**31, m - 2**32, m).to(torch.int32)
+
+
+def test_block_sparsity_causal_counts_lower_triangle():
+    tb = 32                                   # N = 4096, block 128: one word per row
+    full = [(i, j) for i in range(tb) for j in range(i + 1)]
+    assert bench.block_sparsity(_mask(1, 2, tb, full), 4096, 128, True) == 0.0
+    # only the diagonal: tb active of tb (tb + 1) / 2 visible blocks
+    diag = [(i, i) for i in range(tb)]
+    got = bench.block_sparsity(_mask(1, 2, tb, diag), 4096, 128, True)
+    assert got == pytest.approx(1.0 - tb / (tb * (tb + 1) / 2))
+
+
+def test_block_sparsity_reads_bit_31_and_second_word():
+    # block 31 sits in the sign bit of word 0; block 32 opens word 1
+    tb = 40
+    m = _mask(1, 1, tb, [(39, 31), (39, 32)])
+    assert int(m[0, 0, 39, 0]) < 0
+    got = bench.block_sparsity(m, 40 * 64, 64, False)
+    assert got == pytest.approx(1.0 - 2 / (tb * tb))
+
+
+def _result(**counters):
+    base = dict(fwd_hist_tiles=0, fwd_refine_tiles=0, fwd_pv_tiles=0,
+                bwd_row_tiles=0, bwd_col_tiles=0)
+    base.update(counters)
+    return {"counters": base}
+
+
+def test_roofline_counts_the_mma_flops_of_each_kernel():
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 7000.0}
+    w = W.ALPHA15_4K                                  # D = 64
+    unit = 2.0 * 128 * 128 * 64
+    r = _result(fwd_hist_tiles=10, fwd_refine_tiles=2, fwd_pv_tiles=5,
+                bwd_row_tiles=7, bwd_col_tiles=9)
+    # forward: S per histogram or refinement tile; S, P.V and G.V per P.V tile
+    f = bench.roofline_for("fwd", 1.0, [w], [r], peaks, "measured", 1)
+    assert f["bound"] == "tensor"
+    assert f["achieved"] == pytest.approx(round((12 + 3 * 5) * unit / 1e-3 / 1e12, 2))
+    assert f["frac"] == pytest.approx(round(f["achieved"] / 1000.0, 4), abs=1e-4)
+    # backward: 3 MMAs per row tile (S, dP, dQ), 4 per column tile (S^T, dP^T, dV, dK)
+    b = bench.roofline_for("bwd_row", 2.0, [w], [r], peaks, "measured", 1)
+    assert b["achieved"] == pytest.approx(round(7 * 3 * unit / 2e-3 / 1e12, 2))
+    c = bench.roofline_for("bwd_col", 2.0, [w], [r], peaks, "measured", 1)
+    assert c["achieved"] == pytest.approx(round(9 * 4 * unit / 2e-3 / 1e12, 2))
+    # points are averaged: two identical points give the same per-launch figure
+    f2 = bench.roofline_for("fwd", 1.0, [w, w], [r, r], peaks, "measured", 1)
+    assert f2["achieved"] == f["achieved"]
+
+
+def test_roofline_without_mma_work_is_memory_bound():
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 7000.0}
+    h = bench.roofline_for("bwd_fp16_copies", 0.03, [W.ALPHA15_4K], [_result()], peaks,
+                           "fallback", 1)
+    assert h["bound"] == "hbm" and h["peak"] == 7000.0 and h["achieved"] is None
+
+
+def test_source_hash_ignores_comments_only():
+    a = "int f(int x) {  // the answer\n  return x + 1; /* add one */ }\n"
+    b = "int f(int x) {\n/* a longer\n   comment */ return x + 1; }  // trailing\n"
+    c = "int f(int x) { return x + 2; }"
+    assert bench._code_only(a) == bench._code_only(b) == "int f(int x) { return x + 1; }"
+    assert bench._code_only(c) != bench._code_only(a)
+    h = bench.kernel_source_hash()
+    assert len(h) == 16 and int(h, 16) >= 0
+
+
+def test_reference_arm_line():
+    class A:
+        steps = 2
+        warmup = 3
+        workload_desc = "tiny"
+    line = bench.run_reference(A, [W.TINY_FP32.with_(N=96)], 0, 1)
+    assert line["impl"] == "reference" and line["dtype"] == "f64"
+    assert line["value"] > 0 and line["higher_is_better"] is True
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert "rows" in cb["sample"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    assert line["config"]["workload"] == "tiny"
+    # the other ranks do no work
+    assert bench.run_reference(A, [W.TINY_FP32.with_(N=96)], 1, 2) is None

@@ -31,6 +31,12 @@
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and runs asynchronously; a return of ENTMAX_OK means the work
  *     was enqueued, not that it finished.
+ *   - Work runs on the calling thread's current CUDA device.  Every pointer
+ *     and the stream must belong to that device.  One process drives one
+ *     device, as with one process per GPU.  Each kernel's shared-memory limit is
+ *     raised once per process, on the device current at the kernel's first
+ *     launch, so calls on a second device from the same process are not
+ *     supported.
  *   - Arguments are validated before anything is enqueued; on an error return
  *     nothing has been launched and no output was touched.
  *   - Conditions found on the device (a row whose probabilities do not sum to

@@ -149,10 +149,13 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, out_dir: str = ""):
         self.idx = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.f = None
+        out_dir = (out_dir or os.environ.get("BENCH_CLOCKS_DIR")
+                   or os.path.join(ROOT, "bench_clocks"))
+        self.path = os.path.join(out_dir, f"clocks_rank{device_index}.csv")
 
     def __enter__(self):
         try:
@@ -162,8 +165,11 @@ class ClockSampler:
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
+        except OSError:
             self.proc = None
+            if self.f is not None:
+                self.f.close()
+                self.f = None
             return self
         # wait (up to 3 s) for the first sample so the timed region is covered
         t0 = time.time()

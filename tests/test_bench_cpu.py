@@ -5,7 +5,8 @@ These cover what the numbers in bench.py's line are made of:
 - block sparsity read from the bit-packed mask;
 - the MMA FLOPs that the tile counters imply for each kernel's roofline;
 - the comment-insensitive hash that keys the measured DRAM traffic;
-- the fields of the reference arm (the oracle on the host cores).
+- the fields of the reference arm (the oracle on the host cores);
+- the clock summary whose throttle reasons decide whether a run is kept.
 """
 
 import os
@@ -120,3 +121,27 @@ def test_reference_arm_line():
     assert line["config"]["workload"] == "tiny"
     # the other ranks do no work
     assert bench.run_reference(A, [W.TINY_FP32.with_(N=96)], 1, 2) is None
+
+
+def test_clock_summary_median_and_throttle_reasons(tmp_path):
+    cs = bench.ClockSampler(0, out_dir=str(tmp_path))
+    rows = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1900, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1950, 1965, 800.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, [N/A], 1965, [N/A], [N/A], [N/A], [N/A], [N/A], [N/A]",
+    ]
+    with open(cs.path, "w") as f:
+        f.write("\n".join(rows) + "\n")
+    cs.proc = object()     # as if nvidia-smi had run
+    s = cs.summary()
+    assert s["sm_mhz"] == 1950.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
+    monkeypatch.setenv("PATH", str(tmp_path))          # no nvidia-smi on the path
+    with bench.ClockSampler(0, out_dir=str(tmp_path / "clocks")) as cs:
+        pass
+    assert cs.proc is None and cs.f is None
+    assert cs.summary()["reasons"] == ["nvidia-smi unavailable"]

@@ -44,11 +44,11 @@ from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
 # package's csrc/ with comments and white space removed); any other code
 # reports traffic as null.
 TRAFFIC = {
-    ("alpha15_4k", "fwd"): {"bytes": 67279872, "src": "d4da4de491e110e1",
+    ("alpha15_4k", "fwd"): {"bytes": 67279872, "src": "2bc7b14096ef91cb",
                             "from": "profiles/dram_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_row"): {"bytes": 105892608, "src": "d4da4de491e110e1",
+    ("alpha15_4k", "bwd_row"): {"bytes": 105892608, "src": "2bc7b14096ef91cb",
                                 "from": "profiles/dram_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_col"): {"bytes": 72186880, "src": "d4da4de491e110e1",
+    ("alpha15_4k", "bwd_col"): {"bytes": 72186880, "src": "2bc7b14096ef91cb",
                                 "from": "profiles/dram_alpha15_n4096_d64_t1.md (t = 1 launch)"},
 }
 

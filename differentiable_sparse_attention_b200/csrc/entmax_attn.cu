@@ -431,6 +431,8 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, 
   if (!q || !k || !v || !out || !tau || !mask) return ENTMAX_E_NULL;
   int rc = check_common(B, H, N, D, dtype, alpha, block);
   if (rc != ENTMAX_OK) return rc;
+  // only the bf16 kernel runs from the fixed scratch; fp32 inputs take entmax_attn_fwd
+  if (dtype != ENTMAX_DTYPE_BF16) return ENTMAX_E_UNSUPPORTED;
   if (max_iter < 0 || max_iter > ENTMAX_MAX_ITER) return ENTMAX_E_MAXITER;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(tau) ||
       !aligned16(mask))

@@ -124,7 +124,7 @@ size_t entmax_attn_workspace_size(int B, int H, int N, int D, int block, int cau
  *   causal       in   nonzero: key c is visible to query r iff c <= r.
  *   block        in   block size of the mask (64 or 128), rows and keys alike.
  *   max_iter     in   at most this many refinement passes after the histogram
- *                     bound (0..8).  A row stops once its threshold is
+ *                     bound (0..ENTMAX_MAX_ITER).  A row stops once its threshold is
  *                     certified exact -- the step did not cross any score of
  *                     the current support, so the closed-form root on that
  *                     support is tau* -- and a 128-row tile stops once all of
@@ -159,8 +159,9 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
  * allocator).  The paper has no counterpart to this entry point; it exists
  * only for such callers.
  *
- * It runs the kernel of entmax_attn_fwd with the same arguments and outputs
- * (no tau_trace): tau and the mask are the same, and O differs only in the
+ * It runs the bf16 kernel of entmax_attn_fwd with the same arguments and
+ * outputs (no tau_trace; dtype must be ENTMAX_DTYPE_BF16, fp32 returns
+ * ENTMAX_E_UNSUPPORTED): tau and the mask are the same, and O differs only in the
  * rounding of P, which is bf16 here (it multiplies v itself, as no fp16 copy
  * of v fits the scratch) instead of fp16.  It forms no g-weighted means, so
  * entmax_attn_bwd cannot follow it.  Its scratch -- status word, work counters

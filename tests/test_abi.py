@@ -119,3 +119,39 @@ def test_wait_selftest_validation(lib):
     assert lib.entmax_attn_wait_selftest(FAKE, FAKE, 0, None) == dsa.E_SHAPE
     assert lib.entmax_attn_wait_selftest(FAKE, FAKE, 2_000_000_000, None) == dsa.E_SHAPE
     assert lib.entmax_attn_wait_selftest(MISALIGNED, FAKE, 1000, None) == dsa.E_ALIGN
+
+
+def test_grid_size_limit(lib):
+    # one CTA per (batch, head, 128-row tile): B * H * ceil(N / 128) must fit 31 bits
+    assert fwd(lib, B=1 << 14, H=1 << 14, N=1024, ws_bytes=1 << 40) == dsa.E_SHAPE
+    assert fwd(lib, B=1 << 14, H=1 << 13, N=1024, ws_bytes=0) == dsa.E_WORKSPACE
+
+
+def noalloc(lib, *, q=FAKE, B=1, H=1, N=256, D=64, dtype=0, alpha=1.5, causal=1, block=128,
+            max_iter=2, out=FAKE):
+    return lib.entmax_attn_fwd_noalloc(q, FAKE, FAKE, B, H, N, D, dtype, alpha, causal, block,
+                                       max_iter, out, FAKE, FAKE, None)
+
+
+def test_noalloc_argument_validation(lib):
+    assert noalloc(lib, q=None) == dsa.E_NULL
+    assert noalloc(lib, out=None) == dsa.E_NULL
+    assert noalloc(lib, N=0) == dsa.E_SHAPE
+    assert noalloc(lib, D=96) == dsa.E_UNSUPPORTED
+    # fp32 inputs take the workspace forward: the fixed scratch serves bf16 only
+    assert noalloc(lib, dtype=1) == dsa.E_UNSUPPORTED
+    assert noalloc(lib, alpha=3.5) == dsa.E_ALPHA
+    assert noalloc(lib, max_iter=17) == dsa.E_MAXITER
+    assert noalloc(lib, q=MISALIGNED) == dsa.E_ALIGN
+
+
+def test_noalloc_scratch_limit(lib):
+    # causal scratch: 256 + B*H*T(T+1)/2*512 bytes against 8 MiB, T = ceil(N / 128)
+    t = 181
+    assert 256 + t * (t + 1) // 2 * 512 > dsa.NOALLOC_SCRATCH_BYTES
+    assert 256 + (t - 1) * t // 2 * 512 <= dsa.NOALLOC_SCRATCH_BYTES
+    assert noalloc(lib, N=t * 128) == dsa.E_SCRATCH
+    assert noalloc(lib, N=262144) == dsa.E_SCRATCH
+    assert noalloc(lib, B=2, H=16, N=8192) == dsa.E_SCRATCH
+    # non-causal keeps all T^2 tile maxima: T = 128 already exceeds 8 MiB
+    assert noalloc(lib, N=128 * 128, causal=0) == dsa.E_SCRATCH

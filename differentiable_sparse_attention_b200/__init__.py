@@ -124,6 +124,30 @@ def _check_qkv(*ts):
         raise ValueError(f"unsupported dtype {ref.dtype}")
 
 
+_MASK_DTYPES = tuple(d for d in (torch.int32, getattr(torch, "uint32", None)) if d is not None)
+
+
+def _check_buf(name, t, shape, dtypes, device):
+    """A caller-supplied buffer must match what the kernels write or read: the
+    library only sees its pointer, so a smaller or strided buffer would be
+    accessed out of bounds on the device."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    dtypes = dtypes if isinstance(dtypes, tuple) else (dtypes,)
+    if (tuple(t.shape) != tuple(shape) or t.dtype not in dtypes or t.device != device
+            or not t.is_contiguous()):
+        raise ValueError(
+            f"{name} must be a contiguous {'/'.join(str(d) for d in dtypes)} tensor of shape "
+            f"{tuple(shape)} on {device}; got {t.dtype} {tuple(t.shape)} on {t.device}"
+            f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _check_workspace(ws, device):
+    if (not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8 or ws.dim() != 1
+            or ws.device != device or not ws.is_contiguous()):
+        raise ValueError(f"workspace must be a contiguous 1-D uint8 tensor on {device}")
+
+
 class FwdResult(NamedTuple):
     out: torch.Tensor
     tau: torch.Tensor
@@ -159,6 +183,10 @@ def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = True, block: int
         workspace = alloc_workspace(B, H, N, D, block, causal, dev)
     trace_t = (torch.empty((max_iter + 1, B, H, N), dtype=torch.float32, device=dev)
                if trace else None)
+    _check_buf("out", out, q.shape, q.dtype, dev)
+    _check_buf("tau", tau, (B, H, N), torch.float32, dev)
+    _check_buf("mask", mask, (B, H, mrows, mask_words(N, block)), _MASK_DTYPES, dev)
+    _check_workspace(workspace, dev)
     rc = _lib().entmax_attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), B, H, N, D, DTYPE_CODES[q.dtype], float(alpha),
         int(bool(causal)), int(block), int(max_iter), _ptr(out), _ptr(tau), _ptr(mask),
@@ -186,6 +214,12 @@ def entmax_attn_bwd(q, k, v, dout, tau, mask, alpha: float = 1.5, causal: bool =
         if q.dtype == torch.bfloat16:
             raise ValueError("entmax_attn_bwd: bf16 needs the forward's workspace")
         workspace = alloc_workspace(B, H, N, D, block, causal, dev)
+    mrows = (N + block - 1) // block
+    _check_buf("tau", tau, (B, H, N), torch.float32, dev)
+    _check_buf("mask", mask, (B, H, mrows, mask_words(N, block)), _MASK_DTYPES, dev)
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_buf(name, t, q.shape, q.dtype, dev)
+    _check_workspace(workspace, dev)
     rc = _lib().entmax_attn_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(tau), _ptr(mask), B, H, N, D,
         DTYPE_CODES[q.dtype], float(alpha), int(bool(causal)), int(block), _ptr(dq), _ptr(dk),

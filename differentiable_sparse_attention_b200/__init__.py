@@ -304,8 +304,12 @@ def dash_route(q, k, chunk: int, gamma: float, alpha: float = 1.5, max_iter=None
     q: [B, Hq, N, D] bf16, k: [B, Hkv, N, D] bf16, Hq a multiple of Hkv."""
     if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
         raise TypeError("dash_route: q and k must be bfloat16")
+    if int(chunk) < 1:
+        raise ValueError("dash_route: chunk must be at least 1")
     if not (q.is_cuda and k.is_cuda and q.is_contiguous() and k.is_contiguous()):
         raise ValueError("dash_route: q and k must be contiguous CUDA tensors")
+    if q.device != k.device:
+        raise ValueError("dash_route: q and k must live on one CUDA device")
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
     if k.shape != (B, Hkv, N, D):

@@ -96,3 +96,13 @@ def test_backward_checks_its_buffers(cpu_binding):
     with pytest.raises(ValueError, match="workspace"):
         dsa.entmax_attn_bwd(q, k, v, do, f["tau"], f["mask"], 1.5, True, 128,
                             dq=ok["dq"], dk=ok["dk"], dv=ok["dv"])
+
+
+def test_router_rejects_bad_chunk_and_dtype():
+    q = torch.zeros((1, 2, 64, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="chunk"):
+        dsa.dash_route(q, q, 0, 4.0)
+    with pytest.raises(TypeError, match="bfloat16"):
+        dsa.dash_route(q.float(), q.float(), 16, 4.0)
+    with pytest.raises(ValueError, match="CUDA"):     # CPU tensors never reach the library
+        dsa.dash_route(q, q, 16, 4.0)

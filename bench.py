@@ -72,6 +72,13 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+# The two workloads' metrics; every line of an arm, its cpu_baseline and its e2e
+# object use the same unit.
+METRIC = "fwd+bwd alpha-entmax attn ms/step & effective TFLOP/s vs block sparsity, 1 B200"
+UNIT = "effective TFLOP/s (dense-equivalent causal 7*B*H*N^2*D per fwd+bwd step)"
+ROUTER_METRIC = "DashAttention stage-1 entmax router ms/call & logit TFLOP/s, 1 B200"
+ROUTER_UNIT = "logit TFLOP/s (2*B*Hq*N*C*D per call)"
+
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 
@@ -408,9 +415,9 @@ def run_ours(args, points, rank, world, device):
                             f"counters report; peak = 128 lanes x 148 SMs x {sm_mhz:g} MHz"}
 
     line = {
-        "metric": "fwd+bwd alpha-entmax attn ms/step & effective TFLOP/s vs block sparsity, 1 B200",
+        "metric": METRIC,
         "value": round(value, 3),
-        "unit": "effective TFLOP/s (dense-equivalent causal 7*B*H*N^2*D per fwd+bwd step)",
+        "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": round(total_ms / n_steps_all, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -500,7 +507,7 @@ def oracle_sample(w, n_rows: int):
 def cpu_baseline(points):
     w = points[0]
     eff, wall, cores, nr = oracle_sample(w, 2048)
-    return {"value": round(eff / wall / 1e12, 8), "unit": "effective TFLOP/s", "cores": cores,
+    return {"value": round(eff / wall / 1e12, 8), "unit": UNIT, "cores": cores,
             "kind": "oracle", "sample": f"{w.name} t={w.temperature}: {nr} of {w.N} query rows "
             f"(evenly spread) of batch 0 head 0 (1 of {w.B * w.H} heads), fwd+bwd in float64 "
             f"NumPy, {wall:.1f} s wall"}
@@ -525,18 +532,18 @@ def run_reference(args, points, rank, world):
     value = total_eff / total_s / 1e12
     return {
         "impl": "reference",
-        "metric": "fwd+bwd alpha-entmax attn ms/step & effective TFLOP/s vs block sparsity, 1 B200",
+        "metric": METRIC,
         "value": round(value, 8),
-        "unit": "effective TFLOP/s (dense-equivalent causal 7*B*H*N^2*D per fwd+bwd step)",
+        "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_s * 1e3 / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload_desc,
                    "sample": "each step = 256 evenly spread query rows of batch 0 head 0 of one "
                              "sweep point, fwd+bwd through the float64 oracle on host cores"},
-        "cpu_baseline": {"value": round(value, 8), "unit": "effective TFLOP/s", "cores": cores,
+        "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": cores,
                          "kind": "oracle", "sample": "; ".join(samples)},
-        "e2e": {"value": round(value, 8), "unit": "effective TFLOP/s", "h2d_bytes_per_step": 0,
+        "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
 
@@ -591,8 +598,8 @@ def run_router(args, rank, world, device):
     mma_flop = 2 * 2.0 * w["B"] * w["Hq"] * tr * 128 * cp * w["D"]
     achieved = mma_flop / (ms_step * 1e-3) / 1e12
     line = {
-        "metric": "DashAttention stage-1 entmax router ms/call & logit TFLOP/s, 1 B200",
-        "value": round(value, 3), "unit": "logit TFLOP/s (2*B*Hq*N*C*D per call)",
+        "metric": ROUTER_METRIC,
+        "value": round(value, 3), "unit": ROUTER_UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) q, k)",
@@ -640,15 +647,15 @@ def run_router_reference(args, world):
     sample = (f"{rows.size} evenly spread rows x {G} query heads of KV head 0 per step "
               f"({args.steps} steps, {wall:.1f} s)")
     return {"impl": "reference",
-            "metric": "DashAttention stage-1 entmax router ms/call & logit TFLOP/s, 1 B200",
-            "value": round(value, 8), "unit": "logit TFLOP/s (2*B*Hq*N*C*D per call)",
+            "metric": ROUTER_METRIC,
+            "value": round(value, 8), "unit": ROUTER_UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(wall * 1e3 / args.steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "dash_router_16k (oracle sample)", "sample": sample},
-            "cpu_baseline": {"value": round(value, 8), "unit": "logit TFLOP/s", "cores": cores,
+            "cpu_baseline": {"value": round(value, 8), "unit": ROUTER_UNIT, "cores": cores,
                              "kind": "oracle", "sample": sample},
-            "e2e": {"value": round(value, 8), "unit": "logit TFLOP/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": round(value, 8), "unit": ROUTER_UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 

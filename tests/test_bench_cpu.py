@@ -118,6 +118,10 @@ def test_reference_arm_line():
     e2e = line["e2e"]
     assert e2e["value"] == line["value"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    # one metric and one unit for the line, its cpu_baseline and its e2e, the same
+    # as the GPU arm's
+    assert line["metric"] == bench.METRIC
+    assert line["unit"] == cb["unit"] == e2e["unit"] == bench.UNIT
     assert line["config"]["workload"] == "tiny"
     # the other ranks do no work
     assert bench.run_reference(A, [W.TINY_FP32.with_(N=96)], 1, 2) is None
@@ -145,3 +149,52 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
         pass
     assert cs.proc is None and cs.f is None
     assert cs.summary()["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_reference_arm_as_the_driver_runs_it():
+    import json
+    import subprocess
+    run = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert run.returncode == 0, run.stderr[-2000:]
+    lines = [ln for ln in run.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["steps"] == 1 and line["warmup"] == 3
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["config"]["workload"].startswith("alpha15_4k")
+
+
+def test_cpu_baseline_of_the_gpu_arm_uses_the_line_unit():
+    cb = bench.cpu_baseline([W.TINY_FP32.with_(N=96)])
+    assert cb["unit"] == bench.UNIT and cb["kind"] == "oracle" and cb["value"] > 0
+
+
+def test_every_global_name_of_bench_resolves():
+    """The GPU legs of bench.py (run_ours, run_router) do not run here; check
+    statically that every global name any function of bench.py reads is defined,
+    so that a misspelt name cannot first show up on the GPU."""
+    import builtins
+    import symtable
+
+    with open(bench.__file__) as f:
+        top = symtable.symtable(f.read(), bench.__file__, "exec")
+
+    def scopes(t):
+        yield t
+        for c in t.get_children():
+            yield from scopes(c)
+
+    missing = set()
+    checked = 0
+    for t in scopes(top):
+        if str(t.get_type()).lower().split(".")[-1] != "function":
+            continue
+        checked += 1
+        for sym in t.get_symbols():
+            if sym.is_global() and sym.is_referenced():
+                name = sym.get_name()
+                if name not in vars(bench) and not hasattr(builtins, name):
+                    missing.add((t.get_name(), name))
+    assert checked > 10 and missing == set()

@@ -149,6 +149,36 @@ def block_sparsity(mask: torch.Tensor, n: int, block: int, causal: bool) -> floa
     return 1.0 - active / total
 
 
+def visible_blocks(w) -> int:
+    """Blocks of the mask a query block can see: B*H*T(T+1)/2 causal, B*H*T^2 not."""
+    tb = (w.N + w.block - 1) // w.block
+    return w.B * w.H * (tb * (tb + 1) // 2 if w.causal else tb * tb)
+
+
+def active_blocks(w, sparsity: float) -> int:
+    return int(round((1.0 - sparsity) * visible_blocks(w)))
+
+
+def active_block_fit(rows):
+    """Least-squares fit of ms/step = a * visible blocks + b * active blocks over
+    the sweep points: a is the time per block of the dense tau passes (every
+    visible block), b per active block of the sparse passes (P.V and the
+    backward).  None unless the points determine both (two points whose
+    active fraction differs)."""
+    if len(rows) < 2:
+        return None
+    A = np.array([[r["visible_blocks"], r["active_blocks"]] for r in rows], dtype=np.float64)
+    y = np.array([r["ms_per_step"] for r in rows], dtype=np.float64)
+    if (A.max(axis=0) <= 0).any() or np.linalg.matrix_rank(A / A.max(axis=0), tol=1e-3) < 2:
+        return None
+    (a, b), *_ = np.linalg.lstsq(A, y, rcond=None)
+    resid = np.abs(A @ np.array([a, b]) - y) / y
+    return {"model": "ms/step = a * visible blocks + b * active blocks",
+            "a_us_per_visible_block": round(float(a) * 1e3, 6),
+            "b_us_per_active_block": round(float(b) * 1e3, 6),
+            "max_rel_residual": round(float(resid.max()), 4), "points": len(rows)}
+
+
 class ClockSampler:
     """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
 
@@ -371,6 +401,7 @@ def run_ours(args, points, rank, world, device):
         results.append({
             "point": w.name, "temperature": w.temperature, "alpha": w.alpha, "N": N,
             "block": w.block, "block_sparsity": round(sparsity, 4),
+            "visible_blocks": visible_blocks(w), "active_blocks": active_blocks(w, sparsity),
             "ms_per_step": round(ms_step, 4),
             "eff_tflops": round(eff / (ms_step * 1e-3) / 1e12 * world, 2),
             "phases_ms": {n: round(v / args.steps, 4) for n, v in phases.items()},
@@ -433,6 +464,9 @@ def run_ours(args, points, rank, world, device):
         "gpu_launches": kernel_launches,
         "clocks": merge_clocks([r["clocks"] for r in results]),
     }
+    fit = active_block_fit(results)
+    if fit is not None:
+        line["fit"] = fit
     if not args.no_e2e:
         line["e2e"] = {"value": round(total_eff / (e2e_ms * 1e-3) / 1e12, 3),
                        "unit": line["unit"], "h2d_bytes_per_step": h2d // len(points),

@@ -210,3 +210,31 @@ def test_every_global_name_resolves(path):
                 if name not in defined and not hasattr(builtins, name):
                     missing.add((t.get_name(), name))
     assert missing == set()
+
+
+def test_block_counts_of_a_point():
+    w = W.ALPHA15_4K                                    # 32 x 32 blocks of 128, causal
+    assert bench.visible_blocks(w) == 2 * 16 * 32 * 33 // 2
+    assert bench.visible_blocks(w.with_(causal=False)) == 2 * 16 * 32 * 32
+    assert bench.active_blocks(w, 0.0) == bench.visible_blocks(w)
+    assert bench.active_blocks(w, 0.25) == round(0.75 * bench.visible_blocks(w))
+
+
+def test_active_block_fit():
+    def row(w, sparsity, a_us, b_us):
+        vis, act = bench.visible_blocks(w), bench.active_blocks(w, sparsity)
+        return {"visible_blocks": vis, "active_blocks": act,
+                "ms_per_step": (a_us * vis + b_us * act) * 1e-3}
+    long64 = W.long_sweep_point(65536, 1.5)
+    long128 = W.long_sweep_point(131072, 1.5)
+    rows = [row(long64, 0.19, 0.02, 0.05), row(long128, 0.55, 0.02, 0.05),
+            row(W.PLANTED_32K, 0.876, 0.02, 0.05)]
+    fit = bench.active_block_fit(rows)
+    assert fit["a_us_per_visible_block"] == pytest.approx(0.02, rel=1e-4)
+    assert fit["b_us_per_active_block"] == pytest.approx(0.05, rel=1e-4)
+    assert fit["max_rel_residual"] < 1e-4 and fit["points"] == 3
+    # every point at the same active fraction (the 4K sweep at sparsity 0): a and
+    # b cannot be told apart
+    w = W.ALPHA15_4K
+    assert bench.active_block_fit([row(w, 0.0, 0.02, 0.05)] * 3) is None
+    assert bench.active_block_fit([row(long64, 0.19, 0.02, 0.05)]) is None

@@ -18,6 +18,7 @@ from . import dash_router  # noqa: F401
 from .entmax_oracle import (  # noqa: F401
     attention_backward,
     attention_forward,
+    attention_windowed,
     block_margins,
     entmax,
     entmax_jvp,

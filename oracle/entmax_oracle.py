@@ -273,3 +273,121 @@ def attention_backward(q, k, v, dout, alpha: float, causal: bool = True, rows=No
         dk += (dz.T @ q[r]) * scale
         dv += p.T @ dout[r]
     return dq, dk, dv
+
+
+
+def _window_chunk(q, k, v, dout, alpha, causal, block, r, tol, window):
+    """attention_windowed's work for the query rows r (one row block or
+    more, starting on a block boundary): tau, p and dZ on the window entries,
+    their rows of O and dQ, and their contributions to dK and dV."""
+    from scipy import sparse
+
+    n, d = q.shape
+    scale = 1.0 / np.sqrt(d)
+    kend = int(r[-1]) + 1 if causal else n          # keys any row of the chunk sees
+    s = (alpha - 1.0) * scores(q, k[:kend], causal, r)
+    # per row the maximum of each key block (the last one may be partial)
+    nfull = kend // block
+    parts = [s[:, :nfull * block].reshape(r.size, nfull, block).max(axis=-1)]
+    if kend > nfull * block:
+        parts.append(s[:, nfull * block:].max(axis=-1, keepdims=True))
+    bmax = np.concatenate(parts, axis=1) if len(parts) > 1 else parts[0]
+    m = bmax.max(axis=-1)
+    ri, ci = np.nonzero(s > (m - window)[:, None])
+    counts = np.bincount(ri, minlength=r.size)
+    starts = np.concatenate(([0], np.cumsum(counts)[:-1]))
+    pos = np.arange(ri.size) - starts[ri]
+    s_win = np.full((r.size, int(counts.max())), -np.inf)
+    s_win[ri, pos] = s[ri, ci]
+    del s
+    tau = entmax_threshold(s_win, alpha, tol)
+    p_win = entmax_probs(s_win, tau, alpha)
+    # dP = dO V^T on the window entries
+    dp_win = np.zeros_like(s_win)
+    if ri.size * d < r.size * kend:
+        for e0 in range(0, ri.size, 1 << 16):
+            sl = slice(e0, min(ri.size, e0 + (1 << 16)))
+            dp_win[ri[sl], pos[sl]] = np.einsum("ed,ed->e", dout[r[ri[sl]]], v[ci[sl]])
+    else:
+        dp_win[ri, pos] = (dout[r] @ v[:kend].T)[ri, ci]
+    dz_win = entmax_jvp(p_win, dp_win, alpha)
+    pm = sparse.csr_matrix((p_win[ri, pos], (ri, ci)), shape=(r.size, kend))
+    zm = sparse.csr_matrix((dz_win[ri, pos], (ri, ci)), shape=(r.size, kend))
+    res = {"out": pm @ v[:kend], "rowsum": p_win.sum(axis=-1), "tau": tau,
+           "dq": (zm @ k[:kend]) * scale, "dk": (zm.T @ q[r]) * scale, "dv": pm.T @ dout[r],
+           "kend": kend, "bm": bmax - tau[:, None]}
+    return res
+
+
+def attention_windowed(q, k, v, dout, alpha: float, causal: bool = True, block: int = 128,
+                       rows_per_chunk: int = 0, workers: int = 0, tol: float = 1e-12,
+                       _window: float = 1.0):
+    """Forward AND backward of ONE head, exactly as attention_forward and
+    attention_backward define them, with the threshold solved over the scores
+    of the unit window below each row's maximum only.
+
+    Why this is the same computation: tau* >= m - 1 (the lower end of the
+    bracket of entmax_threshold; the summaries use the same fact when they map
+    the scores into a unit window below the maximum before binning them,
+    zh §2.1, it §2A, ja §2.1, es §2A), and every bisection midpoint lies above
+    m - 1.  A score s <= m - 1 therefore adds [s - tau]_+^k = 0 at every point
+    the bisection evaluates and has p = 0 and g = 0 at tau*: dropping it changes
+    neither tau*, nor p, nor dZ = g (dP - delta).  The remaining entries form a
+    sparse matrix per row chunk, and O = P V, dQ = dZ K / sqrt(d),
+    dK = dZ^T Q / sqrt(d) and dV = P^T dO are sparse-times-dense library
+    products over exactly the entries that can be non-zero.  That makes the
+    full head affordable at 4K-128K keys, where the dense routines run the
+    bisection over all N^2 scores.
+
+    ``_window`` (1, the width the bound gives) exists only so that a test can
+    narrow it and check that the pins notice.
+
+    Row chunks are independent; ``workers`` threads (default: the host's
+    cores, at most 16) take them in turn and each keeps its own dK / dV sums,
+    added at the end.
+
+    Returns a dict with out, tau, rowsum, dq, dk, dv (all rows / keys), the
+    block margins [Tr, Tc] (max s - tau over each block, -inf where a block
+    has no valid entry) and the packed mask.
+    """
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    n, d = q.shape
+    tr = (n + block - 1) // block
+    if rows_per_chunk <= 0:
+        rows_per_chunk = max(block, min(1024, (1 << 23) // max(n, 1)) // block * block)
+    if workers <= 0:
+        workers = max(1, min(16, os.cpu_count() or 1))
+    chunks = [np.arange(r0, min(n, r0 + rows_per_chunk)) for r0 in range(0, n, rows_per_chunk)]
+    out = np.empty((n, d))
+    dq = np.empty((n, d))
+    tau_all = np.empty(n)
+    rowsum = np.empty(n)
+    margin = np.full((tr, tr), -np.inf)
+
+    def run(wid):
+        dk_w = np.zeros((n, d))
+        dv_w = np.zeros((n, d))
+        for ci_ in range(wid, len(chunks), workers):
+            r = chunks[ci_]
+            c = _window_chunk(q, k, v, dout, alpha, causal, block, r, tol, _window)
+            out[r] = c["out"]
+            dq[r] = c["dq"]
+            tau_all[r] = c["tau"]
+            rowsum[r] = c["rowsum"]
+            dk_w[:c["kend"]] += c["dk"]
+            dv_w[:c["kend"]] += c["dv"]
+            bm = c["bm"]
+            for rb in range(int(r[0]) // block, int(r[-1]) // block + 1):
+                sel = (r >= rb * block) & (r < (rb + 1) * block)
+                margin[rb, :bm.shape[1]] = bm[sel].max(axis=0)
+        return dk_w, dv_w
+
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        parts = list(ex.map(run, range(workers)))
+    dk = np.sum([p_[0] for p_ in parts], axis=0)
+    dv = np.sum([p_[1] for p_ in parts], axis=0)
+    return {"out": out, "tau": tau_all, "rowsum": rowsum, "dq": dq, "dk": dk, "dv": dv,
+            "margin": margin, "mask": pack_block_mask(margin > 0.0)}

@@ -293,3 +293,96 @@ def test_sampled_rows_match_full():
     np.testing.assert_allclose(dq_t, dq[tail], atol=1e-12)
     np.testing.assert_allclose(dk_t[250:], dk[250:], atol=1e-12)
     np.testing.assert_allclose(dv_t[250:], dv[250:], atol=1e-12)
+
+
+def test_block_margins_hand_computed():
+    # 4 rows x 4 keys, blocks of 2: margin(i, j) = max over the block of s - tau_row.
+    s = np.array([[0.5, -np.inf, -np.inf, -np.inf],
+                  [0.2, 0.9, -np.inf, -np.inf],
+                  [1.0, 0.3, 0.4, -np.inf],
+                  [0.0, 2.0, 0.6, 0.7]])
+    tau = np.array([0.1, 0.5, 0.8, 1.5])
+    # block (0, 0): max(0.5 - 0.1, 0.2 - 0.5, 0.9 - 0.5) = 0.4
+    # block (0, 1): no valid entry -> -inf
+    # block (1, 0): max(1.0 - 0.8, 0.3 - 0.8, 0.0 - 1.5, 2.0 - 1.5) = 0.5
+    # block (1, 1): max(0.4 - 0.8, 0.6 - 1.5, 0.7 - 1.5) = -0.4
+    want = np.array([[0.4, -np.inf], [0.5, -0.4]])
+    got = O.block_margins(s, tau, 0, 2, 4)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-15)
+    # a ragged tail: 3 keys, the last block holds one key only
+    got3 = O.block_margins(s[:3, :3], tau[:3], 0, 2, 3)
+    np.testing.assert_allclose(got3, np.array([[0.4, -np.inf], [0.2, -0.4]]), rtol=0,
+                               atol=1e-15)
+
+
+WINDOWED_CASES = [
+    # n, d, alpha, causal, block, q scale, rows_per_chunk, workers
+    (1, 8, 1.5, True, 64, 1.0, 0, 1),
+    (200, 16, 1.5, True, 64, 2.0, 64, 3),
+    (300, 16, 2.0, True, 128, 3.0, 128, 2),
+    (300, 16, 1.25, False, 64, 1.0, 0, 4),
+    (517, 8, 3.0, True, 64, 1.5, 192, 2),
+    (256, 16, 1.5, False, 128, 0.3, 128, 1),
+]
+
+
+@pytest.mark.parametrize("case", WINDOWED_CASES, ids=[str(i) for i in range(len(WINDOWED_CASES))])
+def test_windowed_matches_dense_definition(case):
+    n, d, alpha, causal, block, qs, rpc, workers = case
+    rng = np.random.default_rng(n * 7 + d)
+    q = rng.normal(size=(n, d)) * qs
+    k, v, do = (rng.normal(size=(n, d)) for _ in range(3))
+    f = O.attention_forward(q, k, v, alpha, causal, block)
+    dq, dk, dv = O.attention_backward(q, k, v, do, alpha, causal)
+    w = O.attention_windowed(q, k, v, do, alpha, causal, block, rows_per_chunk=rpc,
+                             workers=workers)
+    # both thresholds are within the 1e-12 bisection tolerance of tau*; beyond
+    # alpha = 2, p = t^(1/(alpha-1)) has an unbounded slope where a score
+    # enters the support, so that tolerance shows up amplified in O and dV
+    atol = 1e-10 if alpha <= 2.0 else 1e-8
+    np.testing.assert_allclose(w["tau"], f["tau"], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(w["out"], f["out"], rtol=0, atol=atol)
+    np.testing.assert_allclose(w["rowsum"], 1.0, rtol=0, atol=atol)
+    # gradients for alpha <= 2 only: beyond, g = p^(2-alpha) itself is
+    # unbounded at the edge of the support (the library rejects that case)
+    if alpha <= 2.0:
+        for got, want in ((w["dq"], dq), (w["dk"], dk), (w["dv"], dv)):
+            np.testing.assert_allclose(got, want, rtol=0, atol=atol)
+    fin = np.isfinite(f["margin"])
+    assert np.array_equal(fin, np.isfinite(w["margin"]))
+    np.testing.assert_allclose(w["margin"][fin], f["margin"][fin], rtol=0, atol=1e-11)
+    np.testing.assert_array_equal(w["mask"], f["mask"])
+
+
+def test_windowed_wide_windows_and_ties():
+    # all keys equal: every score sits in the window (the widest case), the
+    # result is uniform attention; planted duplicates give exact ties
+    n, d = 130, 8
+    rng = np.random.default_rng(5)
+    q = rng.normal(size=(n, d))
+    k = np.tile(rng.normal(size=(1, d)), (n, 1))
+    v, do = rng.normal(size=(n, d)), rng.normal(size=(n, d))
+    for alpha in (1.5, 2.0):
+        w = O.attention_windowed(q, k, v, do, alpha, True, 64, workers=2)
+        want = np.cumsum(v, axis=0) / np.arange(1, n + 1)[:, None]
+        np.testing.assert_allclose(w["out"], want, rtol=0, atol=1e-10)
+        dq, dk, dv = O.attention_backward(q, k, v, do, alpha, True)
+        np.testing.assert_allclose(w["dv"], dv, rtol=0, atol=1e-10)
+        np.testing.assert_allclose(w["dk"], dk, rtol=0, atol=1e-10)
+        np.testing.assert_allclose(w["dq"], dq, rtol=0, atol=1e-10)
+
+
+def test_windowed_pin_catches_a_narrower_window():
+    # Mutation check: cutting the window at m - 1/2 instead of m - 1 drops
+    # support entries on this wide-support case, and the comparison with the
+    # dense definition must notice.
+    n, d = 96, 8
+    rng = np.random.default_rng(9)
+    q = rng.normal(size=(n, d)) * 0.3
+    k, v, do = (rng.normal(size=(n, d)) for _ in range(3))
+    f = O.attention_forward(q, k, v, 2.0, True, 32)
+    good = O.attention_windowed(q, k, v, do, 2.0, True, 32, workers=1)
+    bad = O.attention_windowed(q, k, v, do, 2.0, True, 32, workers=1, _window=0.5)
+    np.testing.assert_allclose(good["tau"], f["tau"], rtol=0, atol=1e-11)
+    assert np.abs(bad["tau"] - f["tau"]).max() > 1e-3
+    assert np.abs(bad["out"] - f["out"]).max() > 1e-3

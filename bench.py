@@ -7,11 +7,13 @@ batch of the workload, inputs resident in HBM.  Prints ONE JSON line (rank 0).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 Workloads (seeded synthetic data, see differentiable_sparse_attention_b200/workloads.py):
+  long_sweep      B=1 H=8 D=128 t=4, alpha in {1.5, 2}, N in {65536, 131072}
+                  (the default: the long-context sweep whose points span block
+                  sparsity from about 0.2 to above 0.6, the regime the metric
+                  is about)
   alpha15_4k      B=2 H=16 N=4096 D=64 alpha=1.5 causal, q temperature t in {1, 2, 4}
-                  (the default: the sweep the headline metric is quoted on)
   sparsemax_16k   B=1 H=16 N=16384 D=128 alpha=2 t=3
   planted_32k     B=1 H=8 N=32768 D=128 alpha=1.5, 32 planted key blocks per head
-  long_sweep      B=1 H=8 D=128 t=4, alpha in {1.5, 2}, N in {65536, 131072}
   dash_router_16k DashAttention stage-0/1 router: B=1, 32 query heads over 8 KV heads,
                   N=16384 D=128, chunks of 64 (256 chunks), gamma=16, alpha=1.5
 
@@ -39,18 +41,11 @@ sys.path.insert(0, ROOT)
 
 from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
 
-# DRAM bytes (read + write) per launch from one ncu capture, keyed by workload
-# and kernel, valid only for the kernel code they were taken on (hash of the
-# package's csrc/ with comments and white space removed); any other code
-# reports traffic as null.
-TRAFFIC = {
-    ("alpha15_4k", "fwd"): {"bytes": 67279872, "src": "2bc7b14096ef91cb",
-                            "from": "profiles/dram_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_row"): {"bytes": 105892608, "src": "2bc7b14096ef91cb",
-                                "from": "profiles/dram_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-    ("alpha15_4k", "bwd_col"): {"bytes": 72186880, "src": "2bc7b14096ef91cb",
-                                "from": "profiles/dram_alpha15_n4096_d64_t1.md (t = 1 launch)"},
-}
+# DRAM bytes (read + write) per launch of a kernel from one ncu capture, keyed
+# by (sweep point, kernel) and valid only for the kernel code they were taken
+# on (hash of the package's csrc/ with comments and white space removed); any
+# other code reports traffic as null.
+TRAFFIC = {}
 
 
 def _code_only(text: str) -> str:
@@ -417,11 +412,23 @@ def run_ours(args, points, rank, world, device):
     dom = max(phase_tot, key=phase_tot.get)
     dom_ms = phase_tot[dom] / n_steps_all
     roof = roofline_for(dom, dom_ms, points, results, peaks, peaks_kind, args.steps)
-    tr = TRAFFIC.get((args.workload, dom))
-    if (tr is not None and not args.heads and not args.alpha
-            and tr["src"] == kernel_source_hash()):
-        roof["traffic"] = tr["bytes"]
-        roof["traffic_from"] = tr["from"]
+    src = kernel_source_hash()
+
+    def traffic(point_name, kernel):
+        tr = TRAFFIC.get((point_name, kernel))
+        if tr is None or args.heads or args.alpha or tr["src"] != src:
+            return None
+        return tr["bytes"]
+
+    per_point_traffic = [traffic(r["point"], dom) for r in results]
+    if all(t is not None for t in per_point_traffic):
+        roof["traffic"] = int(round(sum(per_point_traffic) / len(per_point_traffic)))
+    # the same roofline for each sweep point on its own
+    for w, r in zip(points, results):
+        pk = max(r["phases_ms"], key=r["phases_ms"].get)
+        r["roofline"] = roofline_for(pk, r["phases_ms"][pk], [w], [r], peaks, peaks_kind,
+                                     args.steps)
+        r["roofline"]["traffic"] = traffic(r["point"], pk)
 
     # the forward's tau passes are bound by the plain ALU pipes, not the tensor
     # cores: the same kernel against 128 lanes x 148 SMs x the clock
@@ -514,13 +521,30 @@ def roofline_for(kernel, ms, points, results, peaks, peaks_kind, steps):
 
 
 # ---------------------------------------------------------------- oracle legs
+def oracle_rows(n: int, budget: int) -> int:
+    """Query rows of a bounded oracle sample: about ``budget`` scores in all
+    (rows x keys), at least 32 rows and at most n."""
+    return int(min(n, max(32, budget // n)))
+
+
+def blas_threads():
+    """Threads of the BLAS library numpy calls into (None if unknown)."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else None
+    except Exception:  # noqa: BLE001 - optional diagnostics only
+        return None
+
+
 def oracle_sample(w, n_rows: int):
     """Time the float64 oracle on n_rows query rows, spread evenly over
     (batch 0, head 0) of workload w: forward for those rows, then their
     backward (dQ rows and their dK/dV contributions) reusing the forward's tau.
-    Returns (effective FLOP of the sample, wall seconds, cores used = CPU
-    seconds / wall seconds).  A causal row sees on average N/2 keys, so the
-    sample's dense-equivalent work is the head's 7 N^2 D scaled by n_rows / N."""
+    Returns (effective FLOP of the sample, wall seconds, measured parallelism
+    = CPU seconds / wall seconds, rows).  A causal row sees on average N/2
+    keys, so the sample's dense-equivalent work is the head's 7 N^2 D scaled by
+    n_rows / N."""
     import oracle as O
 
     x = W.make_inputs(w.with_(B=1, H=1), device="cpu")
@@ -535,31 +559,34 @@ def oracle_sample(w, n_rows: int):
     r1 = resource.getrusage(resource.RUSAGE_SELF)
     cpu = (r1.ru_utime - r0.ru_utime) + (r1.ru_stime - r0.ru_stime)
     eff = effective_flops(w.with_(B=1, H=1)) * rows.size / w.N
-    return eff, wall, max(1, round(cpu / max(wall, 1e-9))), rows.size
+    return eff, wall, round(cpu / max(wall, 1e-9), 2), rows.size
 
 
 def cpu_baseline(points):
     w = points[0]
-    eff, wall, cores, nr = oracle_sample(w, 2048)
-    return {"value": round(eff / wall / 1e12, 8), "unit": UNIT, "cores": cores,
+    eff, wall, par, nr = oracle_sample(w, oracle_rows(w.N, 1 << 26))
+    return {"value": round(eff / wall / 1e12, 8), "unit": UNIT, "cores": os.cpu_count(),
+            "blas_threads": blas_threads(), "parallelism_measured": par,
             "kind": "oracle", "sample": f"{w.name} t={w.temperature}: {nr} of {w.N} query rows "
             f"(evenly spread) of batch 0 head 0 (1 of {w.B * w.H} heads), fwd+bwd in float64 "
-            f"NumPy, {wall:.1f} s wall"}
+            f"NumPy, {wall:.1f} s wall; cores = os.cpu_count() of the host, BLAS threads as "
+            f"numpy reports them, parallelism = CPU seconds / wall seconds"}
 
 
 def run_reference(args, points, rank, world):
     """The oracle as it stands, timed on the host cores: every step is a bounded
-    sample (256 evenly spread query rows of batch 0 head 0) of one sweep point,
-    cycling through the points."""
+    sample (about 2^24 scores: 256 evenly spread query rows of batch 0 head 0
+    up to N = 65536, 128 at 131072) of one sweep point, cycling through the
+    points."""
     if rank != 0:
         return None
     total_eff = 0.0
     total_s = 0.0
-    cores = 1
+    par = 1.0
     samples = []
     for i in range(args.steps):
         w = points[i % len(points)]
-        eff, wall, cores, nr = oracle_sample(w, 256)
+        eff, wall, par, nr = oracle_sample(w, min(256, oracle_rows(w.N, 1 << 24)))
         total_eff += eff
         total_s += wall
         samples.append(f"{w.name} t={w.temperature} ({nr} rows)")
@@ -573,9 +600,11 @@ def run_reference(args, points, rank, world):
         "ms_per_step": round(total_s * 1e3 / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload_desc,
-                   "sample": "each step = 256 evenly spread query rows of batch 0 head 0 of one "
-                             "sweep point, fwd+bwd through the float64 oracle on host cores"},
-        "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": cores,
+                   "sample": "each step = up to 256 evenly spread query rows (about 2^24 "
+                             "scores) of batch 0 head 0 of one sweep point, fwd+bwd through "
+                             "the float64 oracle on host cores"},
+        "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": os.cpu_count(),
+                         "blas_threads": blas_threads(), "parallelism_measured": par,
                          "kind": "oracle", "sample": "; ".join(samples)},
         "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -675,7 +704,7 @@ def run_router_reference(args, world):
         R.route(q64, k64, w["alpha"], w["gamma"], w["chunk"], rows=rows)
     wall = time.perf_counter() - t0
     r1 = resource.getrusage(resource.RUSAGE_SELF)
-    cores = max(1, round(((r1.ru_utime - r0.ru_utime) + (r1.ru_stime - r0.ru_stime)) / wall))
+    par = round(((r1.ru_utime - r0.ru_utime) + (r1.ru_stime - r0.ru_stime)) / wall, 2)
     flop = 2.0 * G * rows.size * C * w["D"] * args.steps
     value = flop / wall / 1e12
     sample = (f"{rows.size} evenly spread rows x {G} query heads of KV head 0 per step "
@@ -687,8 +716,9 @@ def run_router_reference(args, world):
             "ms_per_step": round(wall * 1e3 / args.steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "dash_router_16k (oracle sample)", "sample": sample},
-            "cpu_baseline": {"value": round(value, 8), "unit": ROUTER_UNIT, "cores": cores,
-                             "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": round(value, 8), "unit": ROUTER_UNIT,
+                             "cores": os.cpu_count(), "blas_threads": blas_threads(),
+                             "parallelism_measured": par, "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 8), "unit": ROUTER_UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -698,7 +728,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="alpha15_4k")
+    ap.add_argument("--workload", default="long_sweep")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

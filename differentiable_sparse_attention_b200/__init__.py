@@ -27,7 +27,8 @@ DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
 EXPORTED = ("entmax_attn_mask_words", "entmax_attn_workspace_size", "entmax_attn_fwd",
             "entmax_attn_bwd", "entmax_attn_status", "entmax_attn_counters",
             "entmax_attn_profile", "entmax_attn_profile_read", "entmax_attn_error_string",
-            "entmax_attn_fwd_noalloc", "entmax_attn_wait_selftest")
+            "entmax_attn_fwd_noalloc", "entmax_attn_noalloc_status",
+            "entmax_attn_wait_selftest")
 # include/dash_route.h: the DashAttention stage-0/1 router
 DASH_EXPORTED = ("dash_route_workspace_size", "dash_route_fwd")
 DASH_MAX_CHUNKS = 256
@@ -76,6 +77,8 @@ def _lib():
     lib.entmax_attn_fwd_noalloc.argtypes = ([vp, vp, vp] + [c_int] * 5
                                             + [c_float, c_int, c_int, c_int] + [vp] * 4)
     lib.entmax_attn_fwd_noalloc.restype = c_int
+    lib.entmax_attn_noalloc_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.entmax_attn_noalloc_status.restype = c_int
     lib.entmax_attn_error_string.argtypes = [c_int]
     lib.entmax_attn_error_string.restype = ctypes.c_char_p
     lib.entmax_attn_wait_selftest.argtypes = [vp, vp, ctypes.c_ulonglong, vp]
@@ -236,6 +239,18 @@ def status(workspace: torch.Tensor, stream=None) -> int:
                                    ctypes.byref(word))
     if rc != OK:
         raise EntmaxError(rc, "entmax_attn_status")
+    return int(word.value)
+
+
+def noalloc_status(device=None, stream=None) -> int:
+    """Synchronise the stream and return the status bits (ST_*) of the last
+    entmax_attn_fwd_noalloc call on ``device`` (default: the current one)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    word = ctypes.c_uint32(0)
+    with torch.cuda.device(dev):
+        rc = _lib().entmax_attn_noalloc_status(_stream_ptr(stream, dev), ctypes.byref(word))
+    if rc != OK:
+        raise EntmaxError(rc, "entmax_attn_noalloc_status")
     return int(word.value)
 
 

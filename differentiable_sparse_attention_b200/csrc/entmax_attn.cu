@@ -124,10 +124,34 @@ void prof_mark(int idx, cudaStream_t st) {
   if (g_prof.on && g_prof.created) cudaEventRecord(g_prof.ev[idx], st);
 }
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device.  The attribute belongs to the (kernel, device) pair, so it is set
+// once per pair: a process may drive several devices.
 template <typename Kernel>
 bool set_smem(Kernel k, size_t bytes) {
-  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(bytes)) == cudaSuccess;
+  static std::mutex mu;
+  static const void* done_kernel[64] = {};
+  static uint64_t done_devices[64][4] = {};   // one bit per device 0..255
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return false;
+  const void* key = reinterpret_cast<const void*>(k);
+  std::lock_guard<std::mutex> lock(mu);
+  int slot = -1;
+  for (int a = 0; a < 64 && slot < 0; ++a) {
+    if (done_kernel[a] == key) slot = a;
+    else if (done_kernel[a] == nullptr) { done_kernel[a] = key; slot = a; }
+  }
+  if (slot < 0) {   // more kernels than slots: set the attribute on every launch
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(bytes)) == cudaSuccess;
+  }
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done_devices[slot][dev >> 6] & bit) return true;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes)) != cudaSuccess)
+    return false;
+  done_devices[slot][dev >> 6] |= bit;
+  return true;
 }
 
 // dst = src in fp16 (exact for bf16 values within the fp16 range; others set
@@ -145,8 +169,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   auto kern = entmax_fwd_kernel<D, NS, AM>;
   constexpr size_t smem = fwd_smem_bytes<D, NS>();
   static_assert(smem <= 232448, "forward kernel shared memory");
-  static bool attr_ok = set_smem(kern, smem);
-  if (!attr_ok) return ENTMAX_E_CUDA;
+  if (!set_smem(kern, smem)) return ENTMAX_E_CUDA;
   const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.tr);
   kern<<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
@@ -158,8 +181,7 @@ int launch_bwd_row(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   auto kern = entmax_bwd_row_kernel<D, NSK, NSV, AM>;
   constexpr size_t smem = bwd_row_smem_bytes<D, NSK, NSV>();
   static_assert(smem <= 232448, "bwd row kernel shared memory");
-  static bool attr_ok = set_smem(kern, smem);
-  if (!attr_ok) return ENTMAX_E_CUDA;
+  if (!set_smem(kern, smem)) return ENTMAX_E_CUDA;
   const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.T);
   kern<<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
@@ -171,8 +193,7 @@ int launch_bwd_col(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   auto kern = entmax_bwd_col_kernel<D, NS, AM>;
   constexpr size_t smem = bwd_col_smem_bytes<D, NS>();
   static_assert(smem <= 232448, "bwd column kernel shared memory");
-  static bool attr_ok = set_smem(kern, smem);
-  if (!attr_ok) return ENTMAX_E_CUDA;
+  if (!set_smem(kern, smem)) return ENTMAX_E_CUDA;
   const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.T);
   kern<<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
@@ -229,17 +250,46 @@ int launch_bwd_any(float alpha, int D, const CUtensorMap& mq, const CUtensorMap&
 constexpr size_t kNoAllocScratchBytes = 8u << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch, resolved once per device (in host code
-// the symbol itself is only a host-side handle, not a device address).
+// Unique id of the calling thread's current context (0 if none): a device's
+// context changes after cudaDeviceReset, and with it every device address.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_ctx == nullptr || get_id == nullptr || get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch on the current device (in host code the
+// symbol itself is only a host-side handle, not a device address).  Looked up
+// with cudaGetSymbolAddress on the first call per device, and again whenever
+// that device's context has changed since (after a cudaDeviceReset).
 void* noalloc_scratch_ptr(int device) {
   static std::mutex mu;
   static void* ptrs[256] = {};
+  static unsigned long long ctx_ids[256] = {};
   if (device < 0 || device >= 256) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (ptrs[device] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (ptrs[device] == nullptr || ctx == 0 || ctx != ctx_ids[device]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
     ptrs[device] = p;
+    ctx_ids[device] = current_context_id();
   }
   return ptrs[device];
 }
@@ -268,8 +318,7 @@ F32Params make_f32_params(int B, int H, int N, int D, float alpha, int causal, i
 template <bool A2>
 int launch_fwd_f32(const F32Params& p, cudaStream_t st) {
   auto kern = entmax_fwd_f32_kernel<A2>;
-  static bool attr_ok = set_smem(kern, kF32CandBytes);
-  if (!attr_ok) return ENTMAX_E_CUDA;
+  if (!set_smem(kern, kF32CandBytes)) return ENTMAX_E_CUDA;
   dim3 grid((p.N + 127) / 128, p.BH);
   kern<<<grid, 128, kF32CandBytes, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
@@ -320,8 +369,7 @@ int launch_dash(const CUtensorMap& mq, const CUtensorMap& mkb, const DashParams&
   auto kern = dash_route_kernel<D, AM>;
   constexpr size_t smem = dash_smem_bytes<D>();
   static_assert(smem <= 232448, "router kernel shared memory");
-  static bool attr_ok = set_smem(kern, smem);
-  if (!attr_ok) return ENTMAX_E_CUDA;
+  if (!set_smem(kern, smem)) return ENTMAX_E_CUDA;
   const unsigned grid = static_cast<unsigned>(p.BHkv) * static_cast<unsigned>(p.tr);
   kern<<<grid, kDashThreads, smem, st>>>(mq, mkb, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
@@ -484,6 +532,19 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, 
   p.am1 = alpha - 1.0f;
 
   return launch_fwd_any(alpha, D, mq, mk, mv, p, st);
+}
+
+int entmax_attn_noalloc_status(void* stream, uint32_t* status) {
+  if (!status) return ENTMAX_E_NULL;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return ENTMAX_E_CUDA;
+  const void* ws = noalloc_scratch_ptr(device);
+  if (ws == nullptr) return ENTMAX_E_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ENTMAX_E_CUDA;
+  if (cudaMemcpy(status, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ENTMAX_E_CUDA;
+  return ENTMAX_OK;
 }
 
 int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dout,

@@ -32,11 +32,9 @@
  *     stream) and runs asynchronously; a return of ENTMAX_OK means the work
  *     was enqueued, not that it finished.
  *   - Work runs on the calling thread's current CUDA device.  Every pointer
- *     and the stream must belong to that device.  One process drives one
- *     device, as with one process per GPU.  Each kernel's shared-memory limit is
- *     raised once per process, on the device current at the kernel's first
- *     launch, so calls on a second device from the same process are not
- *     supported.
+ *     and the stream must belong to that device.  A process may drive several
+ *     devices: each kernel's shared-memory limit is raised once per device,
+ *     on that device's first launch of the kernel.
  *   - Arguments are validated before anything is enqueued; on an error return
  *     nothing has been launched and no output was touched.
  *   - Conditions found on the device (a row whose probabilities do not sum to
@@ -172,19 +170,36 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
  *   - Problems whose scratch exceeds the 8 MiB return ENTMAX_E_SCRATCH and
  *     launch nothing (causal: 256 + B*H*T*(T+1)/2*512 bytes, T = ceil(N/128);
  *     e.g. B*H = 16 at N = 4096 needs 4.3 MB).
- *   - The array's device address is looked up once per device, on the first
- *     call made while that device is current; make that first call before any
- *     stream capture on the device.
+ *   - The array's device address is looked up (cudaGetSymbolAddress) on the
+ *     first call made while a device is current, and looked up again when
+ *     that device's context has changed since (after cudaDeviceReset).  With
+ *     CUDA's lazy module loading (the default) that first lookup may also load
+ *     the library's device code, which is when the driver places the 8 MiB
+ *     array in device memory: a caller that must see no device allocation at
+ *     all during its critical section makes one call (a tiny problem will do)
+ *     during its set-up, and makes the first call on a device before any
+ *     stream capture on it.
  *   - All calls on a device share the one array, which keeps the previous
  *     call's contents; the call clears the parts that must start at zero.
  *     Calls whose kernels may overlap on the GPU (other streams, other host
  *     threads) race on the array: serialise them.
- *   - The status word stays in the library's array and is not reported; use
- *     entmax_attn_fwd when the device status is needed.
+ *   - The device status word (ENTMAX_ST_* bits) stays in the array;
+ *     entmax_attn_noalloc_status reads it.
  */
 int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, int H, int N,
                             int D, int dtype, float alpha, int causal, int block, int max_iter,
                             void* out, float* tau, uint32_t* mask, void* stream);
+
+/*
+ * Status of the last entmax_attn_fwd_noalloc on the current device (no
+ * counterpart on the pages; it belongs to the no-alloc entry point above):
+ * synchronises `stream`, then copies the status word of the fixed scratch
+ * array (ENTMAX_ST_* bits, cleared by each entmax_attn_fwd_noalloc call) to
+ * *status.  Allocates nothing.  Returns ENTMAX_E_CUDA if the stream reported
+ * an error.  Only meaningful once the calls it should cover were enqueued on
+ * `stream` (or have finished): a later call on the device clears the word.
+ */
+int entmax_attn_noalloc_status(void* stream, uint32_t* status);
 
 /*
  * Backward pass over the forward's mask (zh §2.3 and ja §2.3: zero blocks are

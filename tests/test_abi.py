@@ -145,6 +145,10 @@ def test_noalloc_argument_validation(lib):
     assert noalloc(lib, q=MISALIGNED) == dsa.E_ALIGN
 
 
+def test_noalloc_status_argument_validation(lib):
+    assert lib.entmax_attn_noalloc_status(None, None) == dsa.E_NULL
+
+
 def test_noalloc_scratch_limit(lib):
     # causal scratch: 256 + B*H*T(T+1)/2*512 bytes against 8 MiB, T = ceil(N / 128)
     t = 181

@@ -13,7 +13,7 @@ import torch
 import oracle as O
 from differentiable_sparse_attention_b200 import entmax_attn_bwd, entmax_attn_fwd, status
 from differentiable_sparse_attention_b200.workloads import Workload, make_inputs
-from parity import BF16_TOL, bf16_half_ulp, check_forward_head, check_grads_head, to64
+from parity import BF16_TOL, bf16_half_ulp, check_forward_head, check_grads_head, tau_rel_err, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -64,7 +64,7 @@ def test_generic_alpha_4k_sampled(cuda_device):
     ref = O.attention_forward(q, k, v, w.alpha, True, 128, rows=rows)
     assert np.abs(f.out[0, h].float().cpu().numpy()[rows] - ref["out"]).max() <= BF16_TOL["out"]
     tau = f.tau[0, h].cpu().numpy().astype(np.float64)[rows]
-    assert (np.abs(tau - ref["tau"]) / np.maximum(1, np.abs(ref["tau"]))).max() <= 1e-3
+    assert tau_rel_err(tau, ref["tau"]) <= 1e-3
     rq, _, _ = O.attention_backward(q, k, v, do, w.alpha, True, rows=rows, tau=ref["tau"])
     tail = np.arange(4096 - 128, 4096)
     _, rk, rv = O.attention_backward(q, k, v, do, w.alpha, True, rows=tail)

@@ -164,12 +164,24 @@ def test_reference_arm_as_the_driver_runs_it():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["steps"] == 1 and line["warmup"] == 3
     assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
-    assert line["config"]["workload"].startswith("alpha15_4k")
+    assert line["config"]["workload"].startswith("long_sweep")
+    cb = line["cpu_baseline"]
+    assert cb["cores"] == os.cpu_count() and cb["parallelism_measured"] > 0
 
 
 def test_cpu_baseline_of_the_gpu_arm_uses_the_line_unit():
     cb = bench.cpu_baseline([W.TINY_FP32.with_(N=96)])
     assert cb["unit"] == bench.UNIT and cb["kind"] == "oracle" and cb["value"] > 0
+    assert cb["cores"] == os.cpu_count() and cb["parallelism_measured"] > 0
+
+
+def test_oracle_sample_rows_are_bounded():
+    # about 2^26 scores for the GPU arm's baseline, never more rows than N
+    assert bench.oracle_rows(4096, 1 << 26) == 4096
+    assert bench.oracle_rows(65536, 1 << 26) == 1024
+    assert bench.oracle_rows(131072, 1 << 26) == 512
+    assert bench.oracle_rows(131072, 1 << 24) == 128
+    assert bench.oracle_rows(96, 1 << 26) == 96
 
 
 def _gpu_only_sources():

@@ -42,6 +42,7 @@ int main(void) {
   CHECK(entmax_attn_fwd_noalloc(fake, fake, fake, 1, 1, 262144, 64, ENTMAX_DTYPE_BF16, 1.5f, 1,
                                 128, 2, fake, (float*)fake, (uint32_t*)fake, NULL)
         == ENTMAX_E_SCRATCH);
+  CHECK(entmax_attn_noalloc_status(NULL, NULL) == ENTMAX_E_NULL);
   CHECK(dash_route_fwd(fake, fake, 1, 3, 2, 256, 64, 16, 4.0f, 1.5f, 4, (float*)fake,
                        (uint32_t*)fake, (uint32_t*)fake, fake, 1u << 30, NULL) == ENTMAX_E_SHAPE);
   printf("%s\n", entmax_attn_error_string(ENTMAX_E_SCRATCH));

@@ -99,3 +99,64 @@ def test_gradient_check_accepts_exact_and_rejects_planted_errors():
         gs[which][5, 2] += 0.05
         with pytest.raises(AssertionError, match=("dq", "dk", "dv")[which]):
             check_grads_head(as_gpu(*gs), 0, 0, q, k, v, do, 1.5, True)
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_full_head_check_accepts_exact_and_rejects_planted_errors(alpha):
+    from parity import check_full_head
+
+    n, block = 200, 64
+    q, k, v, do = _head(n, alpha=alpha)
+    ref = O.attention_windowed(q, k, v, do, alpha, True, block, workers=1)
+
+    def as_gpu(r):
+        f = _as_gpu_forward(r, n, block)
+        grads = tuple(torch.from_numpy(r[g]).to(torch.bfloat16)[None, None]
+                      for g in ("dq", "dk", "dv"))
+        return f, grads
+
+    f, grads = as_gpu(ref)
+    rec = check_full_head(f, grads, 0, 0, ref, block)
+    assert rec["err_out"] <= 1e-2 and rec["err_tau_rel"] <= 1e-6
+    assert rec["mask_diff_outside_ties"] == 0
+    assert all(rec[g]["excess"] <= 0 for g in ("dq", "dk", "dv"))
+
+    for planted, match in ((("out", 17, 3, 0.05), "err_out"), (("tau", 150, None, None), "err_tau"),
+                           (("dq", 5, 2, 0.05), "dq"), (("dk", 0, 1, 0.05), "dk"),
+                           (("dv", 199, 0, 0.05), "dv")):
+        name, r, c, dlt = planted
+        bad = {key: (val.copy() if isinstance(val, np.ndarray) else val) for key, val in ref.items()}
+        if name == "tau":
+            bad["tau"][r] += 0.01 * max(abs(bad["tau"][r]), 1.0)
+        else:
+            bad[name][r, c] += dlt
+        f, grads = as_gpu(bad)
+        # the mask stays the reference's own
+        f.mask = _as_gpu_forward(ref, n, block).mask
+        with pytest.raises(AssertionError, match=match):
+            check_full_head(f, grads, 0, 0, ref, block)
+
+    # a flipped mask bit far from the tie band
+    i, j = np.argwhere(np.abs(ref["margin"]) > 0.1)[0]
+    words = ref["mask"].copy()
+    words[i, j // 32] ^= np.uint32(1) << np.uint32(j % 32)
+    f, grads = as_gpu({**ref, "mask": words})
+    with pytest.raises(AssertionError, match="mask differs"):
+        check_full_head(f, grads, 0, 0, ref, block)
+
+
+def test_grad_stats_counts_entries_beyond_the_literal_bound():
+    from parity import grad_stats
+
+    want = np.array([[0.5, 10.0, 30.0], [-40.0, 0.01, 1.0]])
+    got = want.copy()
+    got[0, 1] += 0.03          # beyond 2e-2, relative 3e-3 (inside 10's half ulp 0.03125)
+    got[1, 0] -= 0.1           # beyond, relative 2.5e-3
+    got[1, 2] += 0.01          # inside the literal bound
+    st = grad_stats(got, want)
+    assert st["n_over_literal"] == 2
+    assert st["max_rel_over_literal"] == pytest.approx(0.03 / 10.0)
+    assert st["min_ref_over_literal"] == pytest.approx(10.0)
+    assert st["max_abs"] == pytest.approx(0.1)
+    # excess over the bf16 half ulp: 10 -> 0.03 - 2^-5, 40 -> 0.1 - 2^-3, 1 -> 0.01 - 2^-8
+    assert st["excess"] == pytest.approx(0.01 - 2.0 ** -8)

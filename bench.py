@@ -494,7 +494,8 @@ def roofline_for(kernel, ms, points, results, peaks, peaks_kind, steps):
       forward:   (hist + refine tiles) * 2*128*128*D + pv tiles * 3 * 2*128*128*D
                  (S, P.V, G.V)
       bwd row:   row tiles * 3 * 2*128*128*D                    (S, dP, dQ)
-      bwd col:   col tiles * 4 * 2*128*128*D                    (S^T, dP^T, dV, dK)
+      bwd col:   col tiles * 5 * 2*128*128*D      (S^T, dP^T, dV, and dK from the
+                 hi and the lo fp16 part of dS^T)
     """
     fl = 0.0
     for w, r in zip(points, results):
@@ -505,7 +506,7 @@ def roofline_for(kernel, ms, points, results, peaks, peaks_kind, steps):
         elif kernel == "bwd_row":
             fl += c["bwd_row_tiles"] * 3 * unit
         elif kernel == "bwd_col":
-            fl += c["bwd_col_tiles"] * 4 * unit
+            fl += c["bwd_col_tiles"] * 5 * unit
     fl /= len(points)
     if fl == 0.0:
         return {"bound": "hbm", "kernel": kernel, "achieved": None, "peak": peaks["hbm_gbs"],

@@ -16,13 +16,15 @@ from typing import NamedTuple, Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libentmax_attn.so")
+# ENTMAX_ATTN_LIB selects another build of the same library, such as the
+# bounds-checked debug build libentmax_attn_bounds.so (see build.py).
+LIB_PATH = os.environ.get("ENTMAX_ATTN_LIB") or os.path.join(_HERE, "libentmax_attn.so")
 
 OK = 0
 E_NULL, E_ALIGN, E_SHAPE, E_UNSUPPORTED, E_ALPHA, E_WORKSPACE, E_CUDA, E_MAXITER, E_SCRATCH = (
     -1, -2, -3, -4, -5, -6, -7, -8, -9)
 NOALLOC_SCRATCH_BYTES = 8 << 20
-ST_NOT_CONVERGED, ST_TIMEOUT, ST_RANGE = 1, 2, 4
+ST_NOT_CONVERGED, ST_TIMEOUT, ST_RANGE, ST_BOUNDS = 1, 2, 4, 8
 DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
 EXPORTED = ("entmax_attn_mask_words", "entmax_attn_workspace_size", "entmax_attn_fwd",
             "entmax_attn_bwd", "entmax_attn_status", "entmax_attn_counters",

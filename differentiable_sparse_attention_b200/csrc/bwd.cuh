@@ -27,9 +27,12 @@ namespace entmax {
 // tm[bh][i][w]: bit (j % 32) of word w = j / 32 is set iff any block of the
 // (block)-granularity mask inside 128x128 tile (i, j) is set.
 __global__ void tile_mask_kernel(const uint32_t* __restrict__ mask, uint32_t* __restrict__ tm,
-                                 int BH, int T, int block, int mask_rows, int mask_words) {
+                                 int BH, int T, int block, int mask_rows, int mask_words,
+                                 uint32_t* status) {
+  bounds_init(status);
   const int wt = (T + 31) / 32;
   const long long total = static_cast<long long>(BH) * T * wt;
+  const long long mask_total = static_cast<long long>(BH) * mask_rows * mask_words;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int w = static_cast<int>(idx % wt);
@@ -38,7 +41,10 @@ __global__ void tile_mask_kernel(const uint32_t* __restrict__ mask, uint32_t* __
     const uint32_t* mrow = mask + static_cast<size_t>(bh) * mask_rows * mask_words;
     uint32_t out = 0u;
     if (block == kTile) {
-      out = mrow[static_cast<size_t>(i) * mask_words + w];
+      const size_t mi = static_cast<size_t>(i) * mask_words + w;
+      if (in_bounds(w < mask_words && static_cast<long long>(bh) * mask_rows * mask_words +
+                                          static_cast<long long>(mi) < mask_total))
+        out = mrow[mi];
     } else {  // 64: rows 2i, 2i+1 and key blocks 2j, 2j+1
       for (int a = 0; a < 2; ++a) {
         const int r = 2 * i + a;
@@ -47,18 +53,24 @@ __global__ void tile_mask_kernel(const uint32_t* __restrict__ mask, uint32_t* __
           const int j = w * 32 + bit;
           if (j >= T) break;
           const int kb = 2 * j;
-          const uint32_t two = (mrow[static_cast<size_t>(r) * mask_words + (kb >> 5)] >> (kb & 31)) & 3u;
+          const size_t mi = static_cast<size_t>(r) * mask_words + (kb >> 5);
+          if (!in_bounds((kb >> 5) < mask_words && static_cast<long long>(bh) * mask_rows *
+                                                          mask_words + static_cast<long long>(mi) <
+                                                      mask_total))
+            continue;
+          const uint32_t two = (mrow[mi] >> (kb & 31)) & 3u;
           if (two) out |= 1u << bit;
         }
       }
     }
-    tm[idx] = out;
+    if (in_bounds(idx < total)) tm[idx] = out;
   }
 }
 
 // tmt[bh][j][w]: bit (i % 32) of word i / 32 = tm[bh][i] bit j.
 __global__ void tile_mask_t_kernel(const uint32_t* __restrict__ tm, uint32_t* __restrict__ tmt,
-                                   int BH, int T) {
+                                   int BH, int T, uint32_t* status) {
+  bounds_init(status);
   const int wt = (T + 31) / 32;
   const long long total = static_cast<long long>(BH) * T * wt;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
@@ -71,9 +83,11 @@ __global__ void tile_mask_t_kernel(const uint32_t* __restrict__ tm, uint32_t* __
     for (int bit = 0; bit < 32; ++bit) {
       const int i = w * 32 + bit;
       if (i >= T) break;
-      out |= ((base[static_cast<size_t>(i) * wt + (j >> 5)] >> (j & 31)) & 1u) << bit;
+      const size_t ti = static_cast<size_t>(i) * wt + (j >> 5);
+      if (in_bounds(static_cast<long long>(bh) * T * wt + static_cast<long long>(ti) < total))
+        out |= ((base[ti] >> (j & 31)) & 1u) << bit;
     }
-    tmt[idx] = out;
+    if (in_bounds(idx < total)) tmt[idx] = out;
   }
 }
 
@@ -83,6 +97,7 @@ __global__ void tile_mask_t_kernel(const uint32_t* __restrict__ tm, uint32_t* __
 // instead of bf16's 8; |x| > 65504 raises ST_RANGE.
 __global__ void to_fp16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
                                size_t n8, uint32_t* status) {
+  bounds_init(status);
   bool bad = false;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -138,12 +153,13 @@ __device__ __forceinline__ int load_tile_list(const uint32_t* rowbits, int wt, u
     int pos = total + incl - cnt;
     while (word) {
       const int b = __ffs(word) - 1;
-      tiles[pos++] = static_cast<uint16_t>(w * 32 + b);
+      if (in_bounds(pos < kMaxTiles)) tiles[pos] = static_cast<uint16_t>(w * 32 + b);
+      ++pos;
       word &= word - 1u;
     }
     total += __shfl_sync(0xffffffffu, incl, 31);
   }
-  return total;
+  return in_bounds(total <= kMaxTiles) ? total : 0;
 }
 
 // Both backward kernels work in half-tile steps: a 128 x 128 tile is two
@@ -206,6 +222,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
   const int i = P.T - 1 - static_cast<int>(blockIdx.x) / P.BH;
   const int bh = static_cast<int>(blockIdx.x) % P.BH;
+  bounds_init(P.status);
+  // elements of a [BH][N] and a [BH][N][D] tensor (bounds-checked build)
+  const size_t n_rows_all = static_cast<size_t>(P.BH) * P.N;
+  const size_t n_elems_all = n_rows_all * D;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.qdo_full, 1);
@@ -252,7 +272,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       {
         for (int t = 0; t < n && ok; ++t) {
-          const int j = sm.tiles[t];
+          const int j = in_bounds(sm.tiles[t] < P.T) ? sm.tiles[t] : 0;
           {
             const uint32_t slot = kc % NSK, use = kc / NSK;
             if (use > 0 && !mbar_wait(&sm.k_empty[slot], (use - 1) & 1, abort_flag, P.status)) { ok = false; break; }
@@ -352,14 +372,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool row_ok = row < P.N;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const uint32_t t_s = t_lane + 128 * wg, t_dp = t_s + kHalf;
-    const float tau_r = row_ok ? P.tau[static_cast<size_t>(bh) * P.N + row] : INFINITY;
+    const size_t row_idx = static_cast<size_t>(bh) * P.N + row;
+    const float tau_r =
+        row_ok && in_bounds(row_idx < n_rows_all) ? P.tau[row_idx] : INFINITY;
     bool ok = true;
     uint32_t use = 0;   // uses of this warpgroup's S/dP buffer
 
     // delta of the row: warpgroup wg takes dimensions [wg D/2, (wg + 1) D/2)
     {
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      if (row_ok) {
+      if (row_ok && in_bounds(row_idx * D + (wg + 1) * (D / 2) <= n_elems_all)) {
         const size_t off = (static_cast<size_t>(bh) * P.N + row) * D + wg * (D / 2);
         const uint4* dsrc = reinterpret_cast<const uint4*>(P.dout16 + off);
         const float4* vsrc = reinterpret_cast<const float4*>(P.vbar + off);
@@ -381,10 +403,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bwd_epi_bar();
     }
     const float delta = sm.part_delta[0][rl] + sm.part_delta[1][rl];
-    if (row_ok && wg == 0) P.delta[static_cast<size_t>(bh) * P.N + row] = delta;
+    if (row_ok && wg == 0 && in_bounds(row_idx < n_rows_all)) P.delta[row_idx] = delta;
 
     for (int t = 0; t < n; ++t) {
-      const int j = sm.tiles[t];
+      const int j = in_bounds(sm.tiles[t] < P.T) ? sm.tiles[t] : 0;
       ok = mbar_wait(&sm.s_full[wg], use & 1, abort_flag, P.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -442,7 +464,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     tc_fence_after();
-    __nv_bfloat16* dst_row = P.dq + (static_cast<size_t>(bh) * P.N + row) * D;
+    __nv_bfloat16* dst_row = P.dq + row_idx * D;
 #pragma unroll 1
     for (int ch = wg * (D / 64); ch < (wg + 1) * (D / 64); ++ch) {
       uint32_t r[32];
@@ -452,7 +474,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) r[e] = 0u;
       }
-      if (row_ok) {
+      if (row_ok && in_bounds(row_idx * D + ch * 32 + 32 <= n_elems_all)) {
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -528,7 +550,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr uint32_t kIdescS = make_idesc(kTile, kHalf, 0, 0, 0, 0);   // K Q_h^T, V dO_h^T
   constexpr uint32_t kIdescAcc = make_idesc(kTile, D, 0, 0, 0, 1);    // P^T_h dO_h, dS^T_h Q_h
   // TMEM buffer b: S^T at 128 b, dP^T at 128 b + 64; the epilogue overwrites
-  // them with P^T and dS^T (fp16, 32-row chunk c packed into columns 32 c .. + 15)
+  // them with P^T and dS^T (fp16, 32-row chunk c packed into columns 32 c .. + 15).
+  // dS^T is kept as two fp16 parts, hi = fp16(dS) and lo = fp16(dS - hi), the
+  // lo part in columns 32 c + 16 .. + 31 of the dP^T region: dK sums dS over
+  // every row that sees the key (up to N), and one fp16 rounding per term
+  // (relative 2^-11) accumulated that far exceeds the output tolerance where
+  // the terms cancel; hi + lo carry about 22 bits.
   constexpr uint32_t kColDV = 256, kColDK = 256 + D;
 
   const int warp = threadIdx.x >> 5;
@@ -536,6 +563,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // causal: key tile j is seen by T - j row tiles, so small j first
   const int j = static_cast<int>(blockIdx.x) / P.BH;
   const int bh = static_cast<int>(blockIdx.x) % P.BH;
+  bounds_init(P.status);
+  const size_t n_rows_all = static_cast<size_t>(P.BH) * P.N;
+  const size_t n_elems_all = n_rows_all * D;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.kv_full, 1);
@@ -584,7 +614,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     for (int t = 0; t < n && ok; ++t) {
-      const int it = sm.tiles[t];
+      const int it = in_bounds(sm.tiles[t] < P.T) ? sm.tiles[t] : 0;
       const uint32_t slot = qc % NS, use = qc / NS;
       if (use > 0) {
         bool w = true;
@@ -605,8 +635,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int r = lane * 4 + e;
         const int row = it * kTile + r;
         const size_t g = static_cast<size_t>(bh) * P.N + row;
-        sm.tau[slot][r] = row < P.N ? P.tau[g] : INFINITY;
-        sm.delta[slot][r] = row < P.N ? P.delta[g] : 0.0f;
+        const bool g_ok = row < P.N && in_bounds(g < n_rows_all);
+        sm.tau[slot][r] = g_ok ? P.tau[g] : INFINITY;
+        sm.delta[slot][r] = g_ok ? P.delta[g] : 0.0f;
       }
       mbar_arrive(&sm.q_full[slot]);
       ++qc;
@@ -650,8 +681,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint32_t a_col = 128 * h + (kk >> 1) * 32 + (kk & 1) * 8;
           mma_f16_ts(tmem + kColDV, tmem + a_col,
                      smem_desc_sw128(do_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescAcc, acc);
-          mma_f16_ts(tmem + kColDK, tmem + a_col + kHalf,
-                     smem_desc_sw128(q_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescAcc, acc);
+          const uint64_t qd = smem_desc_sw128(q_addr + kk * 16 * 128, kSlabBytes, 1024);
+          mma_f16_ts(tmem + kColDK, tmem + a_col + kHalf, qd, kIdescAcc, acc);        // hi
+          mma_f16_ts(tmem + kColDK, tmem + a_col + kHalf + 16, qd, kIdescAcc, 1u);   // lo
         }
         mma_commit(&sm.pt_empty[h]);
         if (h == 1) mma_commit(&sm.q_empty[slot]);
@@ -680,7 +712,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_s = t_lane + 128 * wg, t_dp = t_s + kHalf;
     bool ok = true;
     for (int t = 0; t < n; ++t) {
-      const int it = sm.tiles[t];
+      const int it = in_bounds(sm.tiles[t] < P.T) ? sm.tiles[t] : 0;
       const uint32_t slot = t % NS;
       ok = mbar_wait(&sm.s_full[wg], t & 1, abort_flag, P.status) &&
            mbar_wait(&sm.q_full[slot], (t / NS) & 1, abort_flag, P.status);
@@ -692,7 +724,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // P^T and dS^T of one 32-row chunk; MASKED (diagonal and tail tiles only)
       // keeps rows in [lo_v, hi_v) of the chunk -- a tile-uniform choice
       auto chunk_pds = [&](auto masked_tag, const int ch, const uint32_t (&rs)[32],
-                           const uint32_t (&rp)[32], uint32_t (&wp)[16], uint32_t (&wd)[16]) {
+                           const uint32_t (&rp)[32], uint32_t (&wp)[16], uint32_t (&wd)[16],
+                           uint32_t (&wl)[16]) {
         constexpr bool MASKED = decltype(masked_tag)::value;
         int lo_v = 0, hi_v = 32;
         if constexpr (MASKED) {
@@ -727,21 +760,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           __half2 a1 = __floats2half2_rn(pp[2], pp[3]);
           __half2 b0 = __floats2half2_rn(dd[0], dd[1]);
           __half2 b1 = __floats2half2_rn(dd[2], dd[3]);
+          const float2 f0 = __half22float2(b0), f1 = __half22float2(b1);
+          __half2 c0 = __floats2half2_rn(dd[0] - f0.x, dd[1] - f0.y);
+          __half2 c1 = __floats2half2_rn(dd[2] - f1.x, dd[3] - f1.y);
           wp[e / 2] = *reinterpret_cast<uint32_t*>(&a0);
           wp[e / 2 + 1] = *reinterpret_cast<uint32_t*>(&a1);
           wd[e / 2] = *reinterpret_cast<uint32_t*>(&b0);
           wd[e / 2 + 1] = *reinterpret_cast<uint32_t*>(&b1);
+          wl[e / 2] = *reinterpret_cast<uint32_t*>(&c0);
+          wl[e / 2 + 1] = *reinterpret_cast<uint32_t*>(&c1);
         }
       };
 #pragma unroll 1
       for (int ch = 0; ch < 2; ++ch) {
         uint32_t rs[32], rp[32];
         tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
-        uint32_t wp[16], wd[16];
-        if (msk) chunk_pds(std::true_type{}, ch, rs, rp, wp, wd);
-        else chunk_pds(std::false_type{}, ch, rs, rp, wp, wd);
-        tmem_st16(t_s + ch * 32, wp);    // P^T over the S^T chunk just read
-        tmem_st16(t_dp + ch * 32, wd);   // dS^T over the dP^T chunk
+        uint32_t wp[16], wd[16], wl[16];
+        if (msk) chunk_pds(std::true_type{}, ch, rs, rp, wp, wd, wl);
+        else chunk_pds(std::false_type{}, ch, rs, rp, wp, wd, wl);
+        tmem_st16(t_s + ch * 32, wp);         // P^T over the S^T chunk just read
+        tmem_st16(t_dp + ch * 32, wd);        // dS^T (hi) over the dP^T chunk
+        tmem_st16(t_dp + ch * 32 + 16, wl);   // dS^T (lo) beside it
       }
       tmem_wait_st();
       tc_fence_before();
@@ -759,7 +798,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // warpgroup 0 stores dV, warpgroup 1 stores dK
     const uint32_t col = wg == 0 ? kColDV : kColDK;
     const float scale = wg == 0 ? 1.0f : P.inv_sqrt_d;
-    __nv_bfloat16* dst_row = (wg == 0 ? P.dv : P.dk) + (static_cast<size_t>(bh) * P.N + key) * D;
+    const size_t key_idx = static_cast<size_t>(bh) * P.N + key;
+    __nv_bfloat16* dst_row = (wg == 0 ? P.dv : P.dk) + key_idx * D;
 #pragma unroll 1
     for (int ch = 0; ch < D / 32; ++ch) {
       uint32_t r[32];
@@ -769,7 +809,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) r[e] = 0u;
       }
-      if (key_ok) {
+      if (key_ok && in_bounds(key_idx * D + ch * 32 + 32 <= n_elems_all)) {
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {

@@ -34,6 +34,7 @@ __device__ __forceinline__ float pow_pos(float t, float e) {
 // flag and ST_TIMEOUT in *status exactly as in the attention kernels, and the
 // kernel returns; result[0] = 1 once it has returned from the wait.
 __global__ void wait_selftest_kernel(uint32_t* status, uint32_t* result, unsigned long long limit_ns) {
+  bounds_init(status);
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -125,12 +126,13 @@ __device__ __forceinline__ int compact_tiles(uint32_t* flags, int nwords, uint16
     int pos = total + incl - cnt;
     while (word) {
       const int b = __ffs(word) - 1;
-      tiles[pos++] = static_cast<uint16_t>(w * 32 + b);
+      if (in_bounds(pos < kMaxTiles)) tiles[pos] = static_cast<uint16_t>(w * 32 + b);
+      ++pos;
       word &= word - 1u;
     }
     total += __shfl_sync(0xffffffffu, incl, 31);
   }
-  return total;
+  return in_bounds(total <= kMaxTiles) ? total : 0;
 }
 
 }  // namespace entmax

@@ -36,8 +36,10 @@ constexpr int kDashWords = kDashMaxChunks / 32;
 // remainder), 0 for C <= c < Cp.  One thread per (bh, c, 8 dims).
 __global__ void dash_chunk_mean_kernel(const __nv_bfloat16* __restrict__ k,
                                        __half* __restrict__ kbar, int BH, int N, int D,
-                                       int chunk, int C, int Cp) {
+                                       int chunk, int C, int Cp, uint32_t* status) {
+  bounds_init(status);
   const size_t part = static_cast<size_t>(BH) * Cp * D;
+  const size_t k_elems = static_cast<size_t>(BH) * N * D;
   const int dv = D / 8;
   const long long total = static_cast<long long>(BH) * Cp * dv;
   const float inv = 1.0f / static_cast<float>(chunk);
@@ -48,8 +50,9 @@ __global__ void dash_chunk_mean_kernel(const __nv_bfloat16* __restrict__ k,
     const int c = static_cast<int>(bc % Cp);
     const int bh = static_cast<int>(bc / Cp);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (c < C) {
-      const __nv_bfloat16* src = k + (static_cast<size_t>(bh) * N + static_cast<size_t>(c) * chunk) * D + d8 * 8;
+    const size_t src_off = (static_cast<size_t>(bh) * N + static_cast<size_t>(c) * chunk) * D + d8 * 8;
+    if (c < C && in_bounds(src_off + static_cast<size_t>(chunk - 1) * D + 8 <= k_elems)) {
+      const __nv_bfloat16* src = k + src_off;
       for (int i = 0; i < chunk; ++i) {
         const uint4 w = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(i) * D);
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
@@ -72,6 +75,7 @@ __global__ void dash_chunk_mean_kernel(const __nv_bfloat16* __restrict__ k,
       lo[h] = *reinterpret_cast<const uint32_t*>(&r);
     }
     const size_t at = (static_cast<size_t>(bh) * Cp + c) * D + d8 * 8;
+    if (!in_bounds(at + 8 <= part)) continue;
     *reinterpret_cast<uint4*>(kbar + at) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(kbar + part + at) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
@@ -123,6 +127,8 @@ __global__ void __launch_bounds__(kDashThreads, 1)
   const int i = static_cast<int>(blockIdx.x) / P.BHkv;
   const int bh = static_cast<int>(blockIdx.x) % P.BHkv;
   const int nct = P.Cp / kTile;
+  bounds_init(P.status);
+  const size_t n_rows_all = static_cast<size_t>(P.BHkv) * P.N;   // rows of wbar / row_mask
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.kv_full, 1);
@@ -327,8 +333,10 @@ __global__ void __launch_bounds__(kDashThreads, 1)
     // supports) and the block mask (OR over the 128 rows)
     if (ok) {
       tc_fence_after();
-      float* wrow = P.wbar + (static_cast<size_t>(bh) * P.N + row) * P.C;
-      uint32_t* mrow = P.row_mask + (static_cast<size_t>(bh) * P.N + row) * P.W;
+      const size_t row_idx = static_cast<size_t>(bh) * P.N + row;
+      const bool row_in = !row_ok || in_bounds(row_idx < n_rows_all);
+      float* wrow = P.wbar + row_idx * P.C;
+      uint32_t* mrow = P.row_mask + row_idx * P.W;
       for (int ch = 0; ch < ncp; ++ch) {
         uint32_t acc[32];
         tmem_ld32(t_lane + kColAcc + ch * 32, acc);
@@ -337,11 +345,11 @@ __global__ void __launch_bounds__(kDashThreads, 1)
         for (int e = 0; e < 32; ++e) {
           const float w = __uint_as_float(acc[e]);
           bits |= (w > 0.0f ? 1u : 0u) << e;
-          if (row_ok && ch * 32 + e < P.C) wrow[ch * 32 + e] = w;
+          if (row_ok && row_in && ch * 32 + e < P.C) wrow[ch * 32 + e] = w;
         }
-        if (row_ok && ch < P.W) mrow[ch] = bits;
+        if (row_ok && row_in && ch < P.W) mrow[ch] = bits;
         const uint32_t wbits = __reduce_or_sync(0xffffffffu, row_ok ? bits : 0u);
-        if (lane == 0 && wbits != 0u) atomicOr(&sm.bmask[ch], wbits);
+        if (lane == 0 && wbits != 0u && in_bounds(ch < kDashWords)) atomicOr(&sm.bmask[ch], wbits);
       }
       // sum of p over the G heads is G within 1e-3 per head
       if (row_ok && nvis > 0 && !(fabsf(rowsum - static_cast<float>(P.G)) <= 1e-3f * P.G))
@@ -351,7 +359,9 @@ __global__ void __launch_bounds__(kDashThreads, 1)
   }
 
   __syncthreads();
-  if (!sm.abort_flag && threadIdx.x < P.W)
+  if (!sm.abort_flag && threadIdx.x < P.W &&
+      in_bounds((static_cast<size_t>(bh) * P.tr + i) * P.W + threadIdx.x <
+                static_cast<size_t>(P.BHkv) * P.tr * P.W))
     P.block_mask[(static_cast<size_t>(bh) * P.tr + i) * P.W + threadIdx.x] =
         threadIdx.x < kDashWords ? sm.bmask[threadIdx.x] : 0u;
   if (sm.abort_flag) {

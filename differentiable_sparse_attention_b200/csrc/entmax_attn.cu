@@ -170,6 +170,15 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   constexpr size_t smem = fwd_smem_bytes<D, NS>();
   static_assert(smem <= 232448, "forward kernel shared memory");
   if (!set_smem(kern, smem)) return ENTMAX_E_CUDA;
+  // the kernel moves registers between its warpgroups: the block must be
+  // launched with at least the sum of the split, or the increase never returns
+  static const bool regs_ok = [&] {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
+    return static_cast<long long>(fa.numRegs) * kFwdThreads >=
+           128LL * kFwdCtlRegs + 256LL * kFwdEpiRegs;
+  }();
+  if (!regs_ok) return ENTMAX_E_CUDA;
   const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.tr);
   kern<<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;
@@ -618,8 +627,9 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
     const long long words = static_cast<long long>(BH) * T * wt;
     const int threads = 256;
     const int grid = static_cast<int>(std::min<long long>((words + threads - 1) / threads, 148 * 16));
-    tile_mask_kernel<<<grid, threads, 0, st>>>(mask, tm, BH, T, block, mask_rows, mask_words);
-    tile_mask_t_kernel<<<grid, threads, 0, st>>>(tm, tmt, BH, T);
+    tile_mask_kernel<<<grid, threads, 0, st>>>(mask, tm, BH, T, block, mask_rows, mask_words,
+                                               status_word);
+    tile_mask_t_kernel<<<grid, threads, 0, st>>>(tm, tmt, BH, T, status_word);
     if (cudaGetLastError() != cudaSuccess) return ENTMAX_E_CUDA;
   }
   prof_mark(EV_BWD_MASK, st);
@@ -734,7 +744,7 @@ int dash_route_fwd(const void* q, const void* k, int B, int Hq, int Hkv, int N, 
     const long long total = static_cast<long long>(B) * Hkv * L.Cp * (D / 8);
     const int grid = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 8));
     dash_chunk_mean_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k), kbar, B * Hkv,
-                                                 N, D, chunk, L.C, L.Cp);
+                                                 N, D, chunk, L.C, L.Cp, status);
   }
   if (cudaGetLastError() != cudaSuccess) return ENTMAX_E_CUDA;
   CUtensorMap mq, mkb;

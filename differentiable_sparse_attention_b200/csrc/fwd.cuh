@@ -287,7 +287,10 @@ __device__ __forceinline__ bool solver_step(double F0, double F1, double F2, flo
   return exact;
 }
 
-constexpr int kFwdThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int kFwdThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 2-3 idle, 4-11 epilogue
+// registers per thread after the split: control warpgroup, epilogue warpgroups
+constexpr int kFwdCtlRegs = 56, kFwdEpiRegs = 224;
+static_assert(128 * kFwdCtlRegs + 256 * kFwdEpiRegs <= kFwdThreads * 168, "register split");
 
 __device__ __forceinline__ void fwd_epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 // The same barrier, returning whether v held for any of the 256 threads.
@@ -416,6 +419,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // Work unit: the latest (longest causal) row tiles first.
   const int i = P.tr - 1 - static_cast<int>(blockIdx.x) / P.BH;
   const int bh = static_cast<int>(blockIdx.x) % P.BH;
+  bounds_init(P.status);
+  // elements of the tile-maxima record, of a [BH][N] and a [BH][N][D] tensor
+  // (bounds-checked build)
+  const size_t tmax_elems =
+      static_cast<size_t>(P.BH) *
+      (P.causal ? static_cast<size_t>(P.tr) * (P.tr + 1) / 2 : static_cast<size_t>(P.tr) * P.tc) *
+      (2 * kTile);
+  const size_t n_rows_all = static_cast<size_t>(P.BH) * P.N;
+  const size_t n_elems_all = n_rows_all * D;
   const int ntc = P.causal ? (i + 1) : P.tc;
 
   if (threadIdx.x == 0) {
@@ -465,12 +477,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   bool q_issued = false, q_waited = false;
 
   // epilogue: warpgroup wg, one query row per thread, key columns [hc0, hc0 + 64)
-  const int wg = warp >= 2 ? (warp - 2) >> 2 : 0;
+  const int wg = warp >= 4 ? (warp - 4) >> 2 : 0;
   const int hc0 = wg * 64;
   const int quad = warp & 3;
   const int rl = quad * 32 + lane;
   const int row = i * kTile + rl;
-  const bool row_ok = (warp >= 2) && row < P.N;
+  const bool row_ok = (warp >= 4) && row < P.N;
   const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
   const int n_valid = P.causal ? min(row + 1, P.N) : P.N;
   float m_raw = -INFINITY;                 // running max of q.k (raw units), this half
@@ -487,7 +499,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // never in the support.
   float* cand_base = reinterpret_cast<float*>(&sm.v[0][0]);
   float* my_cand = cand_base + (wg * kCapH) * kTile + rl;     // slot a at my_cand[a * 128]
-  float* other_cand = cand_base + kCapH * kTile + rl;         // warpgroup 1's slots (read by 0)
+  // slot a of this thread's list (checked against the list's capacity in the
+  // bounds-checked build; an out-of-range read yields -inf, below any bound)
+  auto cand_put = [&](int a, float x) {
+    if (in_bounds(a >= 0 && a < kCapH)) my_cand[a * kTile] = x;
+  };
+  auto cand_get = [&](int a) -> float {
+    return in_bounds(a >= 0 && a < kCapH) ? my_cand[a * kTile] : -INFINITY;
+  };
   int ncand = 0;
   float acc_raw = -INFINITY;
   bool cand_over = false;
@@ -505,7 +524,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   auto trace_store = [&](int it, float val) {
     if (P.tau_trace != nullptr && row_ok && wg == 0 && it <= P.max_iter)
-      P.tau_trace[(static_cast<size_t>(it) * P.BH + bh) * P.N + row] = val;
+      if (in_bounds((static_cast<size_t>(it) * P.BH + bh) * P.N + row <
+                    static_cast<size_t>(P.max_iter + 1) * P.BH * P.N))
+        P.tau_trace[(static_cast<size_t>(it) * P.BH + bh) * P.N + row] = val;
   };
   auto needs_mask = [&](int j) {
     return (P.causal && j == i) || (j * kTile + hc0 + 64 > P.N);
@@ -519,6 +540,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   };
 
+  // Control warpgroup (warps 0-3) and epilogue warpgroups (4-11) run their own
+  // pass loops, so that each compiles under its own register budget; both
+  // meet at the same two block barriers per pass.
+  if (warp < 4) {
+  setmaxnreg_dec<kFwdCtlRegs>();
   for (;;) {
     __syncthreads();
     const int kind = sm.ctl_kind;
@@ -539,7 +565,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tma_load_3d(sm.q + s * kTile * 64, &tm_q, &sm.q_full, s * 64, i * kTile, bh);
         }
         for (int t = 0; t < n && ok; ++t) {
-          const int j = sm.tiles[t];
+          const int j = in_bounds(sm.tiles[t] < P.tc) ? sm.tiles[t] : 0;
           {
             const uint32_t slot = kc % NS, use = kc / NS;
             if (use > 0 && !mbar_wait(&sm.k_empty[slot], (use - 1) & 1, abort_flag, P.status)) {
@@ -641,7 +667,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       __syncwarp();
-    } else {
+    }
+  }
+  } else {
+  setmaxnreg_inc<kFwdEpiRegs>();
+  for (;;) {
+    __syncthreads();
+    const int kind = sm.ctl_kind;
+    const int n = sm.ctl_n;
+    const int aborted = sm.abort_flag;
+    __syncthreads();
+    if (aborted || kind == PASS_DONE) break;
+    {
       // ------------------------------------------------------------ epilogue
       bool ok = true;
       double F0 = 0.0, F1 = 0.0, F2 = 0.0;  // refinement sums at tau_c (this half)
@@ -652,7 +689,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         gsum = 0.0f;
       }
       for (int t = 0; t < n; ++t) {
-        const int j = sm.tiles[t];
+        const int j = in_bounds(sm.tiles[t] < P.tc) ? sm.tiles[t] : 0;
         const uint32_t cur = sc++;
         const uint32_t sb = cur % kNSB;
         ok = mbar_wait(&sm.s_full[sb], (cur / kNSB) & 1, abort_flag, P.status);
@@ -665,13 +702,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (kind == PASS_HIST) {
           float tile_max = -INFINITY;
           float cmx0 = -INFINITY, cmx1 = -INFINITY;
-#pragma unroll 1
+          // both 32-column chunks of this tile half in registers, under one wait;
+          // the histogram pass only reads S, so the buffer goes back to the MMA
+          // warp at once
+          uint32_t rr[2][32];
+          tmem_ld32x2(t_s, rr[0], t_s + 32, rr[1]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+#pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
-            uint32_t r[32];
-            tmem_ld32(t_s + ch * 32, r);
             float v[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rr[ch][e]);
             if (msk) apply_mask(v, j, ch);
             // maxima of the four 8-score groups, then of the chunk (a tree)
             float gm[4];
@@ -747,43 +790,47 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               acc_raw = fmaxf(acc_raw, lb * (lb >= 0.0f ? P.inv_c_dn : P.inv_c));
             }
           }
-#pragma unroll 1
+#pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
             const float cm = ch == 0 ? cmx0 : cmx1;
             const bool want = row_ok && !cand_over && cm > acc_raw;
-            if (!__any_sync(0xffffffffu, want)) continue;
-            uint32_t r[32];
-            tmem_ld32(t_s + ch * 32, r);
             if (!want) continue;
             float v[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rr[ch][e]);
             if (msk) apply_mask(v, j, ch);
             if (ncand + 32 > kCapH) {
               if (prunes < kMaxPrunes) {
                 ++prunes;
                 int kept = 0;
                 for (int a = 0; a < ncand; ++a) {
-                  const float xa = my_cand[a * kTile];
-                  if (xa > acc_raw) my_cand[(kept++) * kTile] = xa;
+                  const float xa = cand_get(a);
+                  if (xa > acc_raw) cand_put(kept++, xa);
                 }
+                // the interleaved appends below want an even count
+                if (kept & 1) cand_put(kept++, -INFINITY);
                 ncand = kept;
               }
               cand_over = ncand + 32 > kCapH;
             }
             if (!cand_over) {
+              // two independent append chains, even and odd key columns, into
+              // interleaved slots; the shorter one is then padded with -inf,
+              // which every reader of the list skips like any score below tau
+              int na = ncand >> 1, nb = ncand >> 1;
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                if (v[e] > acc_raw) my_cand[(ncand++) * kTile] = v[e];
+              for (int e = 0; e < 32; e += 2) {
+                if (v[e] > acc_raw) cand_put(2 * na++, v[e]);
+                if (v[e + 1] > acc_raw) cand_put(2 * nb++ + 1, v[e + 1]);
               }
+              for (; nb < na; ++nb) cand_put(2 * nb + 1, -INFINITY);
+              for (; na < nb; ++na) cand_put(2 * na, -INFINITY);
+              ncand = 2 * na;
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
           const float rec = row_ok ? tile_max * P.c : -INFINITY;
-          P.tmax[tmax_index(bh, i, j, P.tr, P.tc, P.causal) + wg * kTile + rl] =
-              __float2half_ru(rec);
+          const size_t ti = tmax_index(bh, i, j, P.tr, P.tc, P.causal) + wg * kTile + rl;
+          if (in_bounds(ti < tmax_elems)) P.tmax[ti] = __float2half_ru(rec);
         } else if (kind == PASS_COLLECT) {
           // rebuild the lists of the rows that overflowed: exactly the scores above lo
           const float thr = collect ? __double2float_rd(lo / P.c) : INFINITY;
@@ -804,7 +851,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               if (v[e] > thr) {
-                if (ncand < kCapH) my_cand[ncand * kTile] = v[e];
+                if (ncand < kCapH) cand_put(ncand, v[e]);
                 ++ncand;
               }
             }
@@ -861,13 +908,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t pb = pc % kNSB;
           ++pc;
           float part = 0.f, gpart = 0.f;
-#pragma unroll 1
+          // both chunks under one wait; each chunk's P (and G) go back into its
+          // own 32 columns, so no store overlaps a column still to be read
+          uint32_t rr[2][32];
+          tmem_ld32x2(t_s, rr[0], t_s + 32, rr[1]);
+#pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
-            uint32_t r[32];
-            tmem_ld32(t_s + ch * 32, r);
             float v[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rr[ch][e]);
             if (msk) apply_mask(v, j, ch);
             uint32_t w[16], wgt[16];
             // p (and g) of the chunk packed for the tensor core: fp16 P and G with
@@ -954,11 +1003,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t bits = __ballot_sync(0xffffffffu, row_ok && part > 0.f);
           if (lane == 0 && bits != 0u) {
             if (P.block == kTile) {
-              atomicOr(&sm.maskw[0][j >> 5], 1u << (j & 31));
+              if (in_bounds((j >> 5) < kMaxMaskWords))
+                atomicOr(&sm.maskw[0][j >> 5], 1u << (j & 31));
             } else {  // block 64: two mask rows per tile, key block 2 j + wg
               const int h = quad >> 1;
               const int kb = 2 * j + wg;
-              atomicOr(&sm.maskw[h][kb >> 5], 1u << (kb & 31));
+              if (in_bounds((kb >> 5) < kMaxMaskWords))
+                atomicOr(&sm.maskw[h][kb >> 5], 1u << (kb & 31));
             }
           }
         }
@@ -975,14 +1026,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int u = 0; u < kU; ++u) {
             jj[u] = (t + u < n) ? static_cast<int>(sm.tiles[t + u]) : -1;
-            hv[u] = jj[u] >= 0 ? __half2float(P.tmax[tmax_index(bh, i, jj[u], P.tr, P.tc,
-                                                                 P.causal) + wg * kTile + rl])
-                               : -INFINITY;
+            const size_t ti = jj[u] >= 0 ? tmax_index(bh, i, jj[u], P.tr, P.tc, P.causal) +
+                                               wg * kTile + rl
+                                         : 0;
+            hv[u] = jj[u] >= 0 && in_bounds(ti < tmax_elems && jj[u] < P.tc)
+                        ? __half2float(P.tmax[ti])
+                        : -INFINITY;
           }
 #pragma unroll
           for (int u = 0; u < kU; ++u) {
             const uint32_t b = __ballot_sync(0xffffffffu, hv[u] > thr);
-            if (lane == 0 && b != 0u && jj[u] >= 0)
+            if (lane == 0 && b != 0u && jj[u] >= 0 && in_bounds((jj[u] >> 5) < kMaxTiles / 32))
               atomicOr(&sm.flags[jj[u] >> 5], 1u << (jj[u] & 31));
           }
         }
@@ -1015,8 +1069,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const float thr = __double2float_rd(lo_r / P.c);
             int kept = 0;
             for (int a = 0; a < ncand; ++a) {
-              const float xa = my_cand[a * kTile];
-              if (xa > thr) my_cand[(kept++) * kTile] = xa;
+              const float xa = cand_get(a);
+              if (xa > thr) cand_put(kept++, xa);
             }
             ncand = kept;
             if (wg == 0) l_drop = fmax(l_drop, static_cast<double>(thr) * P.c);
@@ -1031,7 +1085,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
               const int e = e0 + a;
-              const float tt = e < nown ? fmaf(my_cand[e * kTile], P.c, -tau_c) : -INFINITY;
+              const float tt = e < nown ? fmaf(cand_get(e), P.c, -tau_c) : -INFINITY;
               const bool in = tt > 0.0f;
               const float tp = fmaxf(tt, 0.0f);
               tmn[a] = in ? fminf(tmn[a], tt) : tmn[a];
@@ -1104,7 +1158,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         fence_proxy_async_smem();
         build_list(lo);
         fwd_epi_bar();
-        if (warp == 2) {
+        if (warp == 4) {
           const int nn = compact_tiles(sm.flags, (ntc + 31) >> 5, sm.tiles);
           if (lane == 0) {
             sm.ctl_n = nn;
@@ -1191,7 +1245,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           cand_over = false;
         }
         next_pass(CNT_HIST_TILES);
-        if (warp == 2 && lane == 0 && sm.ctl_kind == PASS_COLLECT)
+        if (warp == 4 && lane == 0 && sm.ctl_kind == PASS_COLLECT)
           atomicAdd(&P.counters[CNT_CAND_OVERFLOW], 1ull);
       } else if (kind == PASS_COLLECT) {
         if (wg == 1) sm.x1[rl].ncand = ncand;
@@ -1202,7 +1256,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (cand_over) sm.cand_overflow = 2;   // refine this tile over the key tiles
         }
         fwd_epi_bar();
-        if (warp == 2 && lane == 0 && sm.cand_overflow == 1) sm.cand_overflow = 0;
+        if (warp == 4 && lane == 0 && sm.cand_overflow == 1) sm.cand_overflow = 0;
         fwd_epi_bar();
         refine_registers();
         if (wg == 0 && row_ok && !row_done && iter < P.max_iter) sm.not_converged = 1;
@@ -1229,7 +1283,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           trace_store(iter, tau_c);
           if (!row_done && iter < P.max_iter) sm.not_converged = 1;
         }
-        if (warp == 2 && lane == 0) ++sm.ctl_iter;
+        if (warp == 4 && lane == 0) ++sm.ctl_iter;
         publish();
         next_pass(CNT_REFINE_TILES);
       } else {  // PASS_PV: write O, tau, mask
@@ -1242,7 +1296,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         sm.xg[wg][rl] = gsum;
         fwd_epi_bar();
         const float gtot = sm.xg[0][rl] + sm.xg[1][rl];
-        __nv_bfloat16* orow = P.out + (static_cast<size_t>(bh) * P.N + row) * D;
+        const size_t row_idx = static_cast<size_t>(bh) * P.N + row;
+        __nv_bfloat16* orow = P.out + row_idx * D;
         // warpgroup wg stores O columns [wg D/2, (wg + 1) D/2)
 #pragma unroll 1
         for (int ch = wg * (D / 64); ch < (wg + 1) * (D / 64); ++ch) {
@@ -1253,7 +1308,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = 0u;
           }
-          if (row_ok) {
+          if (row_ok && in_bounds(row_idx * D + ch * 32 + 32 <= n_elems_all)) {
             uint32_t w[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -1270,7 +1325,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (gv) {
           // g-weighted means of v: G.V / sum g, columns [wg D/2, (wg + 1) D/2)
           const float inv_g = gtot > 0.0f ? 1.0f / gtot : 0.0f;
-          float* vrow = P.vbar + (static_cast<size_t>(bh) * P.N + row) * D;
+          float* vrow = P.vbar + row_idx * D;
 #pragma unroll 1
           for (int ch = wg * (D / 64); ch < (wg + 1) * (D / 64); ++ch) {
             uint32_t r[32];
@@ -1280,7 +1335,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
               for (int e = 0; e < 32; ++e) r[e] = 0u;
             }
-            if (row_ok) {
+            if (row_ok && in_bounds(row_idx * D + ch * 32 + 32 <= n_elems_all)) {
               float4* dst = reinterpret_cast<float4*>(vrow + ch * 32);
 #pragma unroll
               for (int qd = 0; qd < 8; ++qd)
@@ -1294,7 +1349,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_before();
         if (wg == 0 && row_ok) {
           rowsum += sm.xsum[rl];
-          P.tau[static_cast<size_t>(bh) * P.N + row] = tau_c;
+          if (in_bounds(row_idx < n_rows_all)) P.tau[row_idx] = tau_c;
           // sum p = 1 within 1e-3; for k < 1 (alpha > 2) p = t^k turns a rounding
           // eps of s or tau (2^-23 of their magnitude) into eps^k at the edge of
           // the support, so the check allows 8 such terms
@@ -1306,21 +1361,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (wg == 0)
           for (int it = iter + 1; it <= P.max_iter; ++it) trace_store(it, tau_c);
         const int spr = kTile / P.block;
-        const int et = threadIdx.x - 64;
-        for (int idx = et; idx < spr * P.mask_words; idx += kFwdThreads - 64) {
+        const int et = threadIdx.x - 128;
+        for (int idx = et; idx < spr * P.mask_words; idx += kFwdThreads - 128) {
           const int h = idx / P.mask_words;
           const int w = idx - h * P.mask_words;
           const int mrow = i * spr + h;
-          if (mrow < P.mask_rows)
+          if (mrow < P.mask_rows &&
+              in_bounds(h < 2 && w < kMaxMaskWords &&
+                        (static_cast<size_t>(bh) * P.mask_rows + mrow) * P.mask_words + w <
+                            static_cast<size_t>(P.BH) * P.mask_rows * P.mask_words))
             P.mask[(static_cast<size_t>(bh) * P.mask_rows + mrow) * P.mask_words + w] =
                 sm.maskw[h][w];
         }
-        if (warp == 2 && lane == 0) {
+        if (warp == 4 && lane == 0) {
           sm.ctl_kind = PASS_DONE;
           atomicAdd(&P.counters[CNT_PV_TILES], static_cast<unsigned long long>(n));
         }
       }
     }
+  }
   }
 
   // ---------------- teardown: drain in-flight copies / MMAs after an abort,

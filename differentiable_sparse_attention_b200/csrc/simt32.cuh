@@ -88,6 +88,8 @@ __global__ void __launch_bounds__(128) entmax_fwd_f32_kernel(const F32Params P) 
   const int bh = blockIdx.y;
   const int row = i * 128 + tid;
   const bool row_ok = row < P.N;
+  bounds_init(P.status);
+  const size_t n_rows_all = static_cast<size_t>(P.BH) * P.N;
   const float* qh = P.q + static_cast<size_t>(bh) * P.N * kF32D;
   const float* kh = P.k + static_cast<size_t>(bh) * P.N * kF32D;
   const float* vh = P.v + static_cast<size_t>(bh) * P.N * kF32D;
@@ -110,7 +112,9 @@ __global__ void __launch_bounds__(128) entmax_fwd_f32_kernel(const F32Params P) 
     qr[d + 3] = x.w;
   }
   auto trace_store = [&](int it, float val) {
-    if (P.tau_trace != nullptr && row_ok && it <= P.max_iter)
+    if (P.tau_trace != nullptr && row_ok && it <= P.max_iter &&
+        in_bounds((static_cast<size_t>(it) * P.BH + bh) * P.N + row <
+                  static_cast<size_t>(P.max_iter + 1) * n_rows_all))
       P.tau_trace[(static_cast<size_t>(it) * P.BH + bh) * P.N + row] = val;
   };
   // raw scores q.k of keys key0 .. key0+31 (-inf where not visible)
@@ -350,7 +354,7 @@ __global__ void __launch_bounds__(128) entmax_fwd_f32_kernel(const F32Params P) 
       atomicOr(&maskw[h][kb >> 5], 1u << (kb & 31));
     }
   }
-  if (row_ok) {
+  if (row_ok && in_bounds(static_cast<size_t>(bh) * P.N + row < n_rows_all)) {
     float* orow = P.out + (static_cast<size_t>(bh) * P.N + row) * kF32D;
 #pragma unroll
     for (int d = 0; d < kF32D; d += 4)
@@ -363,7 +367,10 @@ __global__ void __launch_bounds__(128) entmax_fwd_f32_kernel(const F32Params P) 
     const int h = idx / P.mask_words;
     const int w = idx - h * P.mask_words;
     const int mrow = i * spr + h;
-    if (mrow < P.mask_rows)
+    if (mrow < P.mask_rows &&
+        in_bounds(h < 2 && w < kMaxMaskWords &&
+                  (static_cast<size_t>(bh) * P.mask_rows + mrow) * P.mask_words + w <
+                      static_cast<size_t>(P.BH) * P.mask_rows * P.mask_words))
       P.mask[(static_cast<size_t>(bh) * P.mask_rows + mrow) * P.mask_words + w] = maskw[h][w];
   }
 }
@@ -386,7 +393,9 @@ __global__ void __launch_bounds__(128) entmax_bwd_row_f32_kernel(const F32Params
   const int rb = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);
   const int bh = blockIdx.y;
   const int row = rb * 64 + (tid >> 1);
-  const bool row_ok = row < P.N;
+  bounds_init(P.status);
+  const bool row_ok = row < P.N && in_bounds(static_cast<size_t>(bh) * P.N + row <
+                                             static_cast<size_t>(P.BH) * P.N);
   const size_t hoff = static_cast<size_t>(bh) * P.N * kF32D;
   const float* kh = P.k + hoff;
   const float* vh = P.v + hoff;
@@ -453,7 +462,9 @@ __global__ void __launch_bounds__(128) entmax_bwd_col_f32_kernel(const F32Params
   const int cb = blockIdx.x;
   const int bh = blockIdx.y;
   const int key = cb * 64 + (tid >> 1);
-  const bool key_ok = key < P.N;
+  bounds_init(P.status);
+  const bool key_ok = key < P.N && in_bounds(static_cast<size_t>(bh) * P.N + key <
+                                             static_cast<size_t>(P.BH) * P.N);
   const size_t hoff = static_cast<size_t>(bh) * P.N * kF32D;
   float kh[32], vh[32], dk[32], dv[32];
 #pragma unroll

@@ -15,7 +15,52 @@ enum : uint32_t {
   ST_NOT_CONVERGED = 1u << 0,  // some row's sum of p is off 1 by more than 1e-3
   ST_TIMEOUT       = 1u << 1,  // a bounded mbarrier wait gave up (kernel exited early)
   ST_RANGE         = 1u << 2,  // a score left the exactly-binnable range (|s| * n_bins >= 2^21)
+  ST_BOUNDS        = 1u << 3,  // bounds-checked build only: an index fell outside its buffer
 };
+
+// ------------------------------------------------------- bounds-checked build
+// Compiled with -DENTMAX_BOUNDS_CHECK, every shared-memory, tensor-memory and
+// global index the kernels compute is checked against its buffer before the
+// access; a violation ORs ST_BOUNDS into the status word and the access is
+// skipped (a load yields zeros), so the kernel never faults or traps on it.
+// Every thread of a kernel records the status word with bounds_init() before
+// its first check (all write the same pointer into one block-shared slot, so
+// each thread sees a valid pointer without a barrier); the checks read it from
+// there.  The normal build compiles every check away.
+#ifdef ENTMAX_BOUNDS_CHECK
+constexpr bool kBoundsCheck = true;
+__device__ __forceinline__ uint32_t** bounds_status_slot() {
+  __shared__ uint32_t* slot;
+  return &slot;
+}
+__device__ __forceinline__ void bounds_init(uint32_t* status) {
+  *reinterpret_cast<uint32_t* volatile*>(bounds_status_slot()) = status;
+}
+__device__ __forceinline__ bool in_bounds(bool ok) {
+  if (!ok) atomicOr(*bounds_status_slot(), ST_BOUNDS);
+  return ok;
+}
+#else
+constexpr bool kBoundsCheck = false;
+__device__ __forceinline__ void bounds_init(uint32_t*) {}
+__device__ __forceinline__ bool in_bounds(bool) { return true; }
+#endif
+
+// Bytes of shared memory the block was launched with (static + dynamic).
+__device__ __forceinline__ uint32_t total_smem_bytes() {
+  uint32_t r;
+  asm("mov.u32 %0, %%total_smem_size;" : "=r"(r));
+  return r;
+}
+
+// A TMEM access of `ncols` 32-bit columns at taddr (lane in the upper 16 bits,
+// column in the lower) stays inside the 512 columns every kernel allocates and
+// in the lane quadrant of the calling warp (warp id % 4).  Warp-uniform.
+__device__ __forceinline__ bool tmem_window_ok(uint32_t taddr, uint32_t ncols) {
+  const uint32_t col = taddr & 0xFFFFu;
+  const uint32_t lane = taddr >> 16;
+  return col + ncols <= 512u && lane == 32u * ((threadIdx.x >> 5) & 3u);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -98,6 +143,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // first.  Completion is signalled on `bar` through the transaction count.
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y, int z) {
+  // the innermost coordinate must be 16-byte aligned (x a multiple of 8 for
+  // 2-byte elements), the box of 128 rows x 128 B lands inside shared memory on
+  // the 1024-byte boundary of the 128-byte swizzle
+  if (kBoundsCheck && !in_bounds((x & 7) == 0 && x >= 0 && y >= 0 && z >= 0 &&
+                                 (smem_u32(smem_dst) & 1023u) == 0 &&
+                                 smem_u32(smem_dst) + 128u * 128u <= total_smem_bytes() &&
+                                 smem_u32(bar) + 8u <= total_smem_bytes()))
+    return;
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
@@ -136,8 +189,25 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16/f16 inputs, f32 accumulate).
+// The accumulator columns [d, d + N) of an M = 128 MMA (N from the
+// instruction descriptor) inside the allocation, and every shared-memory
+// operand starting inside the block's shared memory.
+__device__ __forceinline__ bool mma_operands_ok(uint32_t d_tmem, uint32_t idesc, uint64_t a_desc,
+                                                bool a_in_smem, uint64_t b_desc) {
+  const uint32_t n = ((idesc >> 17) & 0x3Fu) << 3;
+  const uint32_t smem = total_smem_bytes();
+  const uint32_t a_addr = static_cast<uint32_t>(a_desc & 0x3FFFu) << 4;
+  const uint32_t b_addr = static_cast<uint32_t>(b_desc & 0x3FFFu) << 4;
+  // A in TMEM: a 128 x 16 block of 16-bit values spans 8 columns from lane 0
+  const bool a_ok = a_in_smem ? a_addr < smem
+                              : (static_cast<uint32_t>(a_desc) & 0xFFFFu) + 8u <= 512u &&
+                                    (static_cast<uint32_t>(a_desc) >> 16) == 0u;
+  return (d_tmem & 0xFFFFu) + n <= 512u && (d_tmem >> 16) == 0u && a_ok && b_addr < smem;
+}
+
 __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate) {
+  if (kBoundsCheck && !in_bounds(mma_operands_ok(d_tmem, idesc, a_desc, true, b_desc))) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -150,6 +220,7 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uin
 // (lower K index in the low half).  B stays a shared-memory descriptor.
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate) {
+  if (kBoundsCheck && !in_bounds(mma_operands_ok(d_tmem, idesc, a_tmem, false, b_desc))) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -178,6 +249,11 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  if (kBoundsCheck && !in_bounds(tmem_window_ok(taddr, 32))) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) r[e] = 0u;
+    return;
+  }
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -192,6 +268,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 // lane i of its quadrant).  Complete (tmem_wait_st) before the tensor core
 // reads them.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  if (kBoundsCheck && !in_bounds(tmem_window_ok(taddr, 16))) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
@@ -207,6 +284,11 @@ __device__ __forceinline__ void tmem_wait_st() {
 // Two 32-column loads (e.g. S and dP of the same rows) under one wait.
 __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t (&a)[32], uint32_t tb,
                                             uint32_t (&b)[32]) {
+  if (kBoundsCheck && !in_bounds(tmem_window_ok(ta, 32) && tmem_window_ok(tb, 32))) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) a[e] = b[e] = 0u;
+    return;
+  }
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -248,6 +330,20 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t M, uint32_t N, uint32
   return (1u << 4)              // D format f32
          | (a_fmt << 7) | (b_fmt << 10) | (a_mn << 15) | (b_mn << 16) | ((N >> 3) << 17) |
          ((M >> 4) << 24);
+}
+
+// Warpgroup register reallocation: every warp of the warpgroup executes it.
+// The increases of all warpgroups must fit in the registers the block was
+// launched with, or setmaxnreg.inc waits forever.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 }  // namespace entmax

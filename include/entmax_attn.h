@@ -78,6 +78,8 @@ extern "C" {
 #define ENTMAX_ST_NOT_CONVERGED 1u /* some row's sum of p is off 1 by more than 1e-3 */
 #define ENTMAX_ST_TIMEOUT       2u /* a bounded wait gave up; outputs are not valid   */
 #define ENTMAX_ST_RANGE         4u /* |s| * 8 reached 2^21 somewhere: histogram inexact */
+#define ENTMAX_ST_BOUNDS        8u /* bounds-checked build (-DENTMAX_BOUNDS_CHECK) only: an
+                                      index fell outside its buffer; that access was skipped */
 
 #define ENTMAX_MAX_N    262144
 #define ENTMAX_MAX_ITER 16

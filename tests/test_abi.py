@@ -42,6 +42,17 @@ def test_library_exports_every_declared_symbol(lib):
         assert getattr(lib, name) is not None
 
 
+def test_bounds_checked_build_exports_the_same_boundary():
+    # the debug build (-DENTMAX_BOUNDS_CHECK) is the same C ABI
+    path = build_mod.build(bounds_check=True)
+    assert path.endswith("libentmax_attn_bounds.so")
+    dbg = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert getattr(dbg, name) is not None, name
+    dbg.entmax_attn_error_string.restype = ctypes.c_char_p
+    assert dbg.entmax_attn_error_string(0) == b"success"
+
+
 FAKE = ctypes.c_void_p(1 << 20)          # 256-byte aligned, never dereferenced
 MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
 

@@ -170,15 +170,6 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   constexpr size_t smem = fwd_smem_bytes<D, NS>();
   static_assert(smem <= 232448, "forward kernel shared memory");
   if (!set_smem(kern, smem)) return ENTMAX_E_CUDA;
-  // the kernel moves registers between its warpgroups: the block must be
-  // launched with at least the sum of the split, or the increase never returns
-  static const bool regs_ok = [&] {
-    cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
-    return static_cast<long long>(fa.numRegs) * kFwdThreads >=
-           128LL * kFwdCtlRegs + 256LL * kFwdEpiRegs;
-  }();
-  if (!regs_ok) return ENTMAX_E_CUDA;
   const unsigned grid = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.tr);
   kern<<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ENTMAX_OK : ENTMAX_E_CUDA;

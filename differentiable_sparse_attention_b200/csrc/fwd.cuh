@@ -287,10 +287,7 @@ __device__ __forceinline__ bool solver_step(double F0, double F1, double F2, flo
   return exact;
 }
 
-constexpr int kFwdThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 2-3 idle, 4-11 epilogue
-// registers per thread after the split: control warpgroup, epilogue warpgroups
-constexpr int kFwdCtlRegs = 56, kFwdEpiRegs = 224;
-static_assert(128 * kFwdCtlRegs + 256 * kFwdEpiRegs <= kFwdThreads * 168, "register split");
+constexpr int kFwdThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 
 __device__ __forceinline__ void fwd_epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 // The same barrier, returning whether v held for any of the 256 threads.
@@ -477,12 +474,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   bool q_issued = false, q_waited = false;
 
   // epilogue: warpgroup wg, one query row per thread, key columns [hc0, hc0 + 64)
-  const int wg = warp >= 4 ? (warp - 4) >> 2 : 0;
+  const int wg = warp >= 2 ? (warp - 2) >> 2 : 0;
   const int hc0 = wg * 64;
   const int quad = warp & 3;
   const int rl = quad * 32 + lane;
   const int row = i * kTile + rl;
-  const bool row_ok = (warp >= 4) && row < P.N;
+  const bool row_ok = (warp >= 2) && row < P.N;
   const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
   const int n_valid = P.causal ? min(row + 1, P.N) : P.N;
   float m_raw = -INFINITY;                 // running max of q.k (raw units), this half
@@ -525,7 +522,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   auto trace_store = [&](int it, float val) {
     if (P.tau_trace != nullptr && row_ok && wg == 0 && it <= P.max_iter)
       if (in_bounds((static_cast<size_t>(it) * P.BH + bh) * P.N + row <
-                    static_cast<size_t>(P.max_iter + 1) * P.BH * P.N))
+                    static_cast<size_t>(P.max_iter + 1) * n_rows_all))
         P.tau_trace[(static_cast<size_t>(it) * P.BH + bh) * P.N + row] = val;
   };
   auto needs_mask = [&](int j) {
@@ -540,11 +537,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   };
 
-  // Control warpgroup (warps 0-3) and epilogue warpgroups (4-11) run their own
-  // pass loops, so that each compiles under its own register budget; both
-  // meet at the same two block barriers per pass.
-  if (warp < 4) {
-  setmaxnreg_dec<kFwdCtlRegs>();
   for (;;) {
     __syncthreads();
     const int kind = sm.ctl_kind;
@@ -667,18 +659,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       __syncwarp();
-    }
-  }
-  } else {
-  setmaxnreg_inc<kFwdEpiRegs>();
-  for (;;) {
-    __syncthreads();
-    const int kind = sm.ctl_kind;
-    const int n = sm.ctl_n;
-    const int aborted = sm.abort_flag;
-    __syncthreads();
-    if (aborted || kind == PASS_DONE) break;
-    {
+    } else {
       // ------------------------------------------------------------ epilogue
       bool ok = true;
       double F0 = 0.0, F1 = 0.0, F2 = 0.0;  // refinement sums at tau_c (this half)
@@ -702,19 +683,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (kind == PASS_HIST) {
           float tile_max = -INFINITY;
           float cmx0 = -INFINITY, cmx1 = -INFINITY;
-          // both 32-column chunks of this tile half in registers, under one wait;
-          // the histogram pass only reads S, so the buffer goes back to the MMA
-          // warp at once
-          uint32_t rr[2][32];
-          tmem_ld32x2(t_s, rr[0], t_s + 32, rr[1]);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
-#pragma unroll
+#pragma unroll 1
           for (int ch = 0; ch < 2; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(t_s + ch * 32, r);
             float v[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rr[ch][e]);
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (msk) apply_mask(v, j, ch);
             // maxima of the four 8-score groups, then of the chunk (a tree)
             float gm[4];
@@ -790,14 +765,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               acc_raw = fmaxf(acc_raw, lb * (lb >= 0.0f ? P.inv_c_dn : P.inv_c));
             }
           }
-#pragma unroll
+#pragma unroll 1
           for (int ch = 0; ch < 2; ++ch) {
             const float cm = ch == 0 ? cmx0 : cmx1;
             const bool want = row_ok && !cand_over && cm > acc_raw;
+            if (!__any_sync(0xffffffffu, want)) continue;
+            uint32_t r[32];
+            tmem_ld32(t_s + ch * 32, r);
             if (!want) continue;
             float v[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rr[ch][e]);
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (msk) apply_mask(v, j, ch);
             if (ncand + 32 > kCapH) {
               if (prunes < kMaxPrunes) {
@@ -807,27 +785,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                   const float xa = cand_get(a);
                   if (xa > acc_raw) cand_put(kept++, xa);
                 }
-                // the interleaved appends below want an even count
-                if (kept & 1) cand_put(kept++, -INFINITY);
                 ncand = kept;
               }
               cand_over = ncand + 32 > kCapH;
             }
             if (!cand_over) {
-              // two independent append chains, even and odd key columns, into
-              // interleaved slots; the shorter one is then padded with -inf,
-              // which every reader of the list skips like any score below tau
-              int na = ncand >> 1, nb = ncand >> 1;
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                if (v[e] > acc_raw) cand_put(2 * na++, v[e]);
-                if (v[e + 1] > acc_raw) cand_put(2 * nb++ + 1, v[e + 1]);
+              for (int e = 0; e < 32; ++e) {
+                if (v[e] > acc_raw) cand_put(ncand++, v[e]);
               }
-              for (; nb < na; ++nb) cand_put(2 * nb + 1, -INFINITY);
-              for (; na < nb; ++na) cand_put(2 * na, -INFINITY);
-              ncand = 2 * na;
             }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
           const float rec = row_ok ? tile_max * P.c : -INFINITY;
           const size_t ti = tmax_index(bh, i, j, P.tr, P.tc, P.causal) + wg * kTile + rl;
           if (in_bounds(ti < tmax_elems)) P.tmax[ti] = __float2half_ru(rec);
@@ -908,15 +879,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t pb = pc % kNSB;
           ++pc;
           float part = 0.f, gpart = 0.f;
-          // both chunks under one wait; each chunk's P (and G) go back into its
-          // own 32 columns, so no store overlaps a column still to be read
-          uint32_t rr[2][32];
-          tmem_ld32x2(t_s, rr[0], t_s + 32, rr[1]);
-#pragma unroll
+#pragma unroll 1
           for (int ch = 0; ch < 2; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(t_s + ch * 32, r);
             float v[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rr[ch][e]);
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
             if (msk) apply_mask(v, j, ch);
             uint32_t w[16], wgt[16];
             // p (and g) of the chunk packed for the tensor core: fp16 P and G with
@@ -1158,7 +1127,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         fence_proxy_async_smem();
         build_list(lo);
         fwd_epi_bar();
-        if (warp == 4) {
+        if (warp == 2) {
           const int nn = compact_tiles(sm.flags, (ntc + 31) >> 5, sm.tiles);
           if (lane == 0) {
             sm.ctl_n = nn;
@@ -1245,7 +1214,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           cand_over = false;
         }
         next_pass(CNT_HIST_TILES);
-        if (warp == 4 && lane == 0 && sm.ctl_kind == PASS_COLLECT)
+        if (warp == 2 && lane == 0 && sm.ctl_kind == PASS_COLLECT)
           atomicAdd(&P.counters[CNT_CAND_OVERFLOW], 1ull);
       } else if (kind == PASS_COLLECT) {
         if (wg == 1) sm.x1[rl].ncand = ncand;
@@ -1256,7 +1225,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (cand_over) sm.cand_overflow = 2;   // refine this tile over the key tiles
         }
         fwd_epi_bar();
-        if (warp == 4 && lane == 0 && sm.cand_overflow == 1) sm.cand_overflow = 0;
+        if (warp == 2 && lane == 0 && sm.cand_overflow == 1) sm.cand_overflow = 0;
         fwd_epi_bar();
         refine_registers();
         if (wg == 0 && row_ok && !row_done && iter < P.max_iter) sm.not_converged = 1;
@@ -1283,7 +1252,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           trace_store(iter, tau_c);
           if (!row_done && iter < P.max_iter) sm.not_converged = 1;
         }
-        if (warp == 4 && lane == 0) ++sm.ctl_iter;
+        if (warp == 2 && lane == 0) ++sm.ctl_iter;
         publish();
         next_pass(CNT_REFINE_TILES);
       } else {  // PASS_PV: write O, tau, mask
@@ -1361,8 +1330,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (wg == 0)
           for (int it = iter + 1; it <= P.max_iter; ++it) trace_store(it, tau_c);
         const int spr = kTile / P.block;
-        const int et = threadIdx.x - 128;
-        for (int idx = et; idx < spr * P.mask_words; idx += kFwdThreads - 128) {
+        const int et = threadIdx.x - 64;
+        for (int idx = et; idx < spr * P.mask_words; idx += kFwdThreads - 64) {
           const int h = idx / P.mask_words;
           const int w = idx - h * P.mask_words;
           const int mrow = i * spr + h;
@@ -1373,13 +1342,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             P.mask[(static_cast<size_t>(bh) * P.mask_rows + mrow) * P.mask_words + w] =
                 sm.maskw[h][w];
         }
-        if (warp == 4 && lane == 0) {
+        if (warp == 2 && lane == 0) {
           sm.ctl_kind = PASS_DONE;
           atomicAdd(&P.counters[CNT_PV_TILES], static_cast<unsigned long long>(n));
         }
       }
     }
-  }
   }
 
   // ---------------- teardown: drain in-flight copies / MMAs after an abort,

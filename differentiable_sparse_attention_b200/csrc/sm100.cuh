@@ -46,12 +46,6 @@ __device__ __forceinline__ void bounds_init(uint32_t*) {}
 __device__ __forceinline__ bool in_bounds(bool) { return true; }
 #endif
 
-// Bytes of shared memory the block was launched with (static + dynamic).
-__device__ __forceinline__ uint32_t total_smem_bytes() {
-  uint32_t r;
-  asm("mov.u32 %0, %%total_smem_size;" : "=r"(r));
-  return r;
-}
 
 // A TMEM access of `ncols` 32-bit columns at taddr (lane in the upper 16 bits,
 // column in the lower) stays inside the 512 columns every kernel allocates and
@@ -64,6 +58,19 @@ __device__ __forceinline__ bool tmem_window_ok(uint32_t taddr, uint32_t ncols) {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Every extern __shared__ array starts at the block's dynamic shared memory.
+extern __shared__ __align__(16) uint8_t entmax_dyn_smem[];
+
+// Shared-window address one past the block's dynamic shared memory (the
+// operands and TMA boxes of these kernels all live there).  The window also
+// holds a reserved area and the static variables below the dynamic part, so
+// the bound is the dynamic base plus its size, not the total size alone.
+__device__ __forceinline__ uint32_t dyn_smem_end() {
+  uint32_t sz;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(sz));
+  return smem_u32(entmax_dyn_smem) + sz;
 }
 
 // ---------------------------------------------------------------- mbarriers
@@ -148,8 +155,9 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
   // the 1024-byte boundary of the 128-byte swizzle
   if (kBoundsCheck && !in_bounds((x & 7) == 0 && x >= 0 && y >= 0 && z >= 0 &&
                                  (smem_u32(smem_dst) & 1023u) == 0 &&
-                                 smem_u32(smem_dst) + 128u * 128u <= total_smem_bytes() &&
-                                 smem_u32(bar) + 8u <= total_smem_bytes()))
+                                 smem_u32(smem_dst) >= smem_u32(entmax_dyn_smem) &&
+                                 smem_u32(smem_dst) + 128u * 128u <= dyn_smem_end() &&
+                                 smem_u32(bar) + 8u <= dyn_smem_end()))
     return;
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
@@ -195,7 +203,7 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ bool mma_operands_ok(uint32_t d_tmem, uint32_t idesc, uint64_t a_desc,
                                                 bool a_in_smem, uint64_t b_desc) {
   const uint32_t n = ((idesc >> 17) & 0x3Fu) << 3;
-  const uint32_t smem = total_smem_bytes();
+  const uint32_t smem = dyn_smem_end();
   const uint32_t a_addr = static_cast<uint32_t>(a_desc & 0x3FFFu) << 4;
   const uint32_t b_addr = static_cast<uint32_t>(b_desc & 0x3FFFu) << 4;
   // A in TMEM: a 128 x 16 block of 16-bit values spans 8 columns from lane 0
@@ -303,6 +311,39 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t (&a)[32], uint
 }
 
 
+// The same two loads issued without waiting; tmem_wait_ld_x2 completes them.
+// Between the two calls the registers hold no data yet: only
+// tmem_wait_ld_x2's outputs may be read.
+__device__ __forceinline__ void tmem_ld32x2_async(uint32_t ta, uint32_t (&a)[32], uint32_t tb,
+                                                  uint32_t (&b)[32]) {
+  if (kBoundsCheck && !in_bounds(tmem_window_ok(ta, 32) && tmem_window_ok(tb, 32))) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) a[e] = b[e] = 0u;
+    return;
+  }
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];"
+      : ENTMAX_R32(a), ENTMAX_R32(b)
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+// Waits for this thread's TMEM loads.  a and b pass through the statement as
+// read-write operands, so the compiler cannot move a use of them above it.
+#define ENTMAX_RW32(r)                                                                       \
+  "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),       \
+      "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), \
+      "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),           \
+      "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),           \
+      "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+__device__ __forceinline__ void tmem_wait_ld_x2(uint32_t (&a)[32], uint32_t (&b)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : ENTMAX_RW32(a), ENTMAX_RW32(b) : : "memory");
+}
+
 // ---------------------------------------------------------------- descriptors
 // UMMA shared-memory matrix descriptor for a 128-byte-swizzled operand whose
 // tile base is 1024-byte aligned.  Fields: start address >> 4 (bits 0-13),
@@ -332,18 +373,5 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t M, uint32_t N, uint32
          ((M >> 4) << 24);
 }
 
-// Warpgroup register reallocation: every warp of the warpgroup executes it.
-// The increases of all warpgroups must fit in the registers the block was
-// launched with, or setmaxnreg.inc waits forever.
-template <int N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
 
 }  // namespace entmax

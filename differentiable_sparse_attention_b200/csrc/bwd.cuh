@@ -220,8 +220,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int i = P.T - 1 - static_cast<int>(blockIdx.x) / P.BH;
-  const int bh = static_cast<int>(blockIdx.x) % P.BH;
+  // head by head (the resident CTAs share one or two heads' K and V in L2),
+  // the longest causal rows first within a head
+  const int i = P.T - 1 - static_cast<int>(blockIdx.x) % P.T;
+  const int bh = static_cast<int>(blockIdx.x) / P.T;
   bounds_init(P.status);
   // elements of a [BH][N] and a [BH][N][D] tensor (bounds-checked build)
   const size_t n_rows_all = static_cast<size_t>(P.BH) * P.N;
@@ -441,14 +443,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           w[e] = *reinterpret_cast<const uint32_t*>(&h2);
         }
       };
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t rs[32], rp[32];
-        tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
-        uint32_t w[16];
-        if (msk) chunk_ds(std::true_type{}, ch, rs, rp, w);
-        else chunk_ds(std::false_type{}, ch, rs, rp, w);
-        tmem_st16(t_s + ch * 32, w);   // dS over the S chunk just read
+      // chunk 1's loads are in flight while chunk 0 is computed and stored
+      {
+        uint32_t rs[2][32], rp[2][32], w[16];
+        tmem_ld32x2(t_s, rs[0], t_dp, rp[0]);
+        tmem_ld32x2_async(t_s + 32, rs[1], t_dp + 32, rp[1]);
+        if (msk) chunk_ds(std::true_type{}, 0, rs[0], rp[0], w);
+        else chunk_ds(std::false_type{}, 0, rs[0], rp[0], w);
+        tmem_st16(t_s, w);             // dS over the S chunk just read
+        tmem_wait_ld_x2(rs[1], rp[1]);
+        if (msk) chunk_ds(std::true_type{}, 1, rs[1], rp[1], w);
+        else chunk_ds(std::false_type{}, 1, rs[1], rp[1], w);
+        tmem_st16(t_s + 32, w);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -560,9 +566,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // causal: key tile j is seen by T - j row tiles, so small j first
-  const int j = static_cast<int>(blockIdx.x) / P.BH;
-  const int bh = static_cast<int>(blockIdx.x) % P.BH;
+  // head by head (the resident CTAs share one or two heads' Q and dO in L2);
+  // causal: key tile j is seen by T - j row tiles, so small j first within a head
+  const int j = static_cast<int>(blockIdx.x) % P.T;
+  const int bh = static_cast<int>(blockIdx.x) / P.T;
   bounds_init(P.status);
   const size_t n_rows_all = static_cast<size_t>(P.BH) * P.N;
   const size_t n_elems_all = n_rows_all * D;
@@ -771,16 +778,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           wl[e / 2 + 1] = *reinterpret_cast<uint32_t*>(&c1);
         }
       };
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t rs[32], rp[32];
-        tmem_ld32x2(t_s + ch * 32, rs, t_dp + ch * 32, rp);
-        uint32_t wp[16], wd[16], wl[16];
-        if (msk) chunk_pds(std::true_type{}, ch, rs, rp, wp, wd, wl);
-        else chunk_pds(std::false_type{}, ch, rs, rp, wp, wd, wl);
-        tmem_st16(t_s + ch * 32, wp);         // P^T over the S^T chunk just read
-        tmem_st16(t_dp + ch * 32, wd);        // dS^T (hi) over the dP^T chunk
-        tmem_st16(t_dp + ch * 32 + 16, wl);   // dS^T (lo) beside it
+      // chunk 1's loads are in flight while chunk 0 is computed and stored
+      {
+        uint32_t rs[2][32], rp[2][32], wp[16], wd[16], wl[16];
+        tmem_ld32x2(t_s, rs[0], t_dp, rp[0]);
+        tmem_ld32x2_async(t_s + 32, rs[1], t_dp + 32, rp[1]);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          if (ch == 1) tmem_wait_ld_x2(rs[1], rp[1]);
+          if (msk) chunk_pds(std::true_type{}, ch, rs[ch], rp[ch], wp, wd, wl);
+          else chunk_pds(std::false_type{}, ch, rs[ch], rp[ch], wp, wd, wl);
+          tmem_st16(t_s + ch * 32, wp);         // P^T over the S^T chunk just read
+          tmem_st16(t_dp + ch * 32, wd);        // dS^T (hi) over the dP^T chunk
+          tmem_st16(t_dp + ch * 32 + 16, wl);   // dS^T (lo) beside it
+        }
       }
       tmem_wait_st();
       tc_fence_before();

@@ -413,9 +413,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Work unit: the latest (longest causal) row tiles first.
-  const int i = P.tr - 1 - static_cast<int>(blockIdx.x) / P.BH;
-  const int bh = static_cast<int>(blockIdx.x) % P.BH;
+  // Work unit: head by head, and within a head the latest (longest causal) row
+  // tiles first.  The CTAs resident at one time then stream the K and V tiles of
+  // one or two heads, which stay in L2, instead of every head's.
+  const int i = P.tr - 1 - static_cast<int>(blockIdx.x) % P.tr;
+  const int bh = static_cast<int>(blockIdx.x) / P.tr;
   bounds_init(P.status);
   // elements of the tile-maxima record, of a [BH][N] and a [BH][N][D] tensor
   // (bounds-checked build)

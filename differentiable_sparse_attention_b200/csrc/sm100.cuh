@@ -344,6 +344,25 @@ __device__ __forceinline__ void tmem_wait_ld_x2(uint32_t (&a)[32], uint32_t (&b)
   asm volatile("tcgen05.wait::ld.sync.aligned;" : ENTMAX_RW32(a), ENTMAX_RW32(b) : : "memory");
 }
 
+// One 32-column load issued without waiting; tmem_wait_ld_x1 completes it.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+  if (kBoundsCheck && !in_bounds(tmem_window_ok(taddr, 32))) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) r[e] = 0u;
+    return;
+  }
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : ENTMAX_R32(r)
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld_x1(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : ENTMAX_RW32(r) : : "memory");
+}
+
 // ---------------------------------------------------------------- descriptors
 // UMMA shared-memory matrix descriptor for a 128-byte-swizzled operand whose
 // tile base is 1024-byte aligned.  Fields: start address >> 4 (bits 0-13),

@@ -416,7 +416,7 @@ def run_ours(args, points, rank, world, device):
 
     def traffic(point_name, kernel):
         tr = TRAFFIC.get((point_name, kernel))
-        if tr is None or args.heads or args.alpha or tr["src"] != src:
+        if tr is None or args.heads or args.alpha or args.block or tr["src"] != src:
             return None
         return tr["bytes"]
 
@@ -737,6 +737,8 @@ def main():
                     help="override H (small cases for profiler captures)")
     ap.add_argument("--alpha", type=float, default=0.0,
                     help="override alpha (any value in [1.05, 3]; 1.5 and 2 have closed forms)")
+    ap.add_argument("--block", type=int, default=0, choices=[0, 64, 128],
+                    help="override the mask block size (the sparsity is then reported at it)")
     args = ap.parse_args()
     if args.workload == "dash_router_16k":
         world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -763,6 +765,8 @@ def main():
         points = [p.with_(H=args.heads) for p in points]
     if args.alpha:
         points = [p.with_(alpha=args.alpha, name=f"{p.name}_as_alpha{args.alpha:g}") for p in points]
+    if args.block:
+        points = [p.with_(block=args.block) for p in points]
     args.workload_desc = (f"{args.workload}: " + ", ".join(
         f"B={p.B} H={p.H} N={p.N} D={p.D} alpha={p.alpha} t={p.temperature}"
         + (f" planted={p.planted_blocks}" if p.planted_blocks else "") for p in points)

@@ -119,6 +119,7 @@ __global__ void to_fp16_kernel(const __nv_bfloat16* __restrict__ src, __half* __
 
 struct BwdParams {
   int BH, N, T, wt;          // T = 128-tiles per side, wt = words per tile-mask row
+  int hg;                    // heads per work group (work_item)
   int causal;
   float c;                   // (alpha - 1) / sqrt(D)
   float inv_sqrt_d;
@@ -220,10 +221,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // head by head (the resident CTAs share one or two heads' K and V in L2),
-  // the longest causal rows first within a head
-  const int i = P.T - 1 - static_cast<int>(blockIdx.x) % P.T;
-  const int bh = static_cast<int>(blockIdx.x) / P.T;
+  // head groups that share L2, the longest causal rows first within a group
+  const WorkItem wi = work_item(static_cast<int>(blockIdx.x), P.BH, P.T, P.hg);
+  const int i = P.T - 1 - wi.r;
+  const int bh = wi.bh;
   bounds_init(P.status);
   // elements of a [BH][N] and a [BH][N][D] tensor (bounds-checked build)
   const size_t n_rows_all = static_cast<size_t>(P.BH) * P.N;
@@ -566,10 +567,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // head by head (the resident CTAs share one or two heads' Q and dO in L2);
-  // causal: key tile j is seen by T - j row tiles, so small j first within a head
-  const int j = static_cast<int>(blockIdx.x) % P.T;
-  const int bh = static_cast<int>(blockIdx.x) / P.T;
+  // head groups that share L2; causal: key tile j is seen by T - j row tiles,
+  // so small j first within a group
+  const WorkItem wi = work_item(static_cast<int>(blockIdx.x), P.BH, P.T, P.hg);
+  const int j = wi.r;
+  const int bh = wi.bh;
   bounds_init(P.status);
   const size_t n_rows_all = static_cast<size_t>(P.BH) * P.N;
   const size_t n_elems_all = n_rows_all * D;

@@ -81,6 +81,24 @@ __device__ __forceinline__ uint64_t shl64(uint64_t x, uint32_t sh) {
   return r;
 }
 
+// Work order of the attention kernels.  Heads run in groups of hg, a group's
+// streamed K and V (or Q and dO) small enough to stay in L2 together; within a
+// group the CTAs take their tile in the order r = 0, 1, ... across the group's
+// heads (r = 0 the longest causal row or column).  Ordering all heads at once
+// lets the resident CTAs span every head, whose tiles then miss L2 at long N;
+// one head at a time unbalances the SMs when a CTA's work is comparable to an
+// SM's share (short N).
+struct WorkItem {
+  int bh;
+  int r;
+};
+__device__ __forceinline__ WorkItem work_item(int block, int BH, int T, int hg) {
+  const int g = block / (hg * T);
+  const int gsize = min(hg, BH - g * hg);
+  const int rem = block - g * hg * T;
+  return {g * hg + rem % gsize, rem / gsize};
+}
+
 // Offset (in elements) of the tile-max record of (row tile i, key tile j) of
 // head bh: two halves (key columns 0-63 and 64-127) of 128 rows each.  Causal
 // problems store only the lower triangle j <= i.

@@ -59,6 +59,15 @@ WsLayout ws_layout(int B, int H, int N, int D, int causal) {
   return L;
 }
 
+// Heads per work group of the attention kernels (work_item): as many as keep
+// the K and V (or Q and dO) tiles they stream, 2 bytes x N x D each, within
+// 64 MB of the 126 MB L2.
+int head_group(int BH, int N, int D) {
+  const double per_head = 4.0 * static_cast<double>(N) * D;
+  const int hg = static_cast<int>((64.0 * 1024 * 1024) / per_head);
+  return std::max(1, std::min(BH, hg));
+}
+
 // ------------------------------------------------------------ argument checks
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -447,6 +456,7 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, int B, int H, i
   p.N = N;
   p.tr = (N + kTile - 1) / kTile;
   p.tc = p.tr;
+  p.hg = head_group(BH, N, D);
   p.causal = causal ? 1 : 0;
   p.block = block;
   p.mask_rows = (N + block - 1) / block;
@@ -510,6 +520,7 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, int B, 
   p.N = N;
   p.tr = (N + kTile - 1) / kTile;
   p.tc = p.tr;
+  p.hg = head_group(BH, N, D);
   p.causal = causal ? 1 : 0;
   p.block = block;
   p.mask_rows = (N + block - 1) / block;
@@ -630,6 +641,7 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
   p.N = N;
   p.T = T;
   p.wt = wt;
+  p.hg = head_group(BH, N, D);
   p.causal = causal ? 1 : 0;
   p.c = (alpha - 1.0f) / std::sqrt(static_cast<float>(D));
   p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(D));

@@ -41,6 +41,7 @@ namespace entmax {
 
 struct FwdParams {
   int BH, N, tr, tc;         // heads x batch, sequence length, 128-tiles per row / column
+  int hg;                    // heads per work group (work_item)
   int causal;
   int block;                 // mask block size, 64 or 128
   int mask_rows, mask_words; // ceil(N / block), words per mask row
@@ -413,11 +414,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Work unit: head by head, and within a head the latest (longest causal) row
-  // tiles first.  The CTAs resident at one time then stream the K and V tiles of
-  // one or two heads, which stay in L2, instead of every head's.
-  const int i = P.tr - 1 - static_cast<int>(blockIdx.x) % P.tr;
-  const int bh = static_cast<int>(blockIdx.x) / P.tr;
+  // Work unit: head groups that share L2, the latest (longest causal) row tiles
+  // first within a group.
+  const WorkItem wi = work_item(static_cast<int>(blockIdx.x), P.BH, P.tr, P.hg);
+  const int i = P.tr - 1 - wi.r;
+  const int bh = wi.bh;
   bounds_init(P.status);
   // elements of the tile-maxima record, of a [BH][N] and a [BH][N][D] tensor
   // (bounds-checked build)

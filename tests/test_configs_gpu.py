@@ -29,7 +29,10 @@ pytestmark = pytest.mark.gpu
 
 POINTS = ([W.ALPHA15_4K.with_(temperature=t) for t in W.ALPHA15_4K_TEMPERATURES]
           + [W.SPARSEMAX_16K, W.PLANTED_32K]
-          + [W.long_sweep_point(n, a) for n, a in W.LONG_SWEEP_POINTS])
+          + [W.long_sweep_point(n, a) for n, a in W.LONG_SWEEP_POINTS]
+          # the 4K sweep's sparsest point with a mask of 64 x 64 blocks, where a 128
+          # x 128 tile often has only one active 64-wide half
+          + [W.ALPHA15_4K.with_(temperature=4.0, block=64, name="alpha1.5_n4096_d64_block64")])
 
 
 @pytest.mark.parametrize("w", POINTS, ids=[f"{p.name}_t{p.temperature}" for p in POINTS])

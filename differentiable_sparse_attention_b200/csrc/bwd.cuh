@@ -298,8 +298,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(&sm.qdo_full, 0, abort_flag, P.status);
+    // every lane runs the issue loop (warp-uniform descriptors); one elected
+    // lane issues each MMA and commit
+    {
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.qdo_full, 0, abort_flag, P.status));
       const uint32_t q_addr = smem_u32(sm.q), do_addr = smem_u32(sm.dout);
       uint32_t step = 0, dstep = 0;     // half-tile steps issued (S/dP) and dQ steps issued
       uint32_t kcm = 0, vcm = 0;        // K / V tiles consumed
@@ -309,28 +311,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t h = step & 1, use = step >> 1;
         const uint32_t ks = kcm % NSK, vs = vcm % NSV;
         if (h == 0) {
-          if (!mbar_wait(&sm.k_full[ks], (kcm / NSK) & 1, abort_flag, P.status)) return false;
-          if (!mbar_wait(&sm.v_full[vs], (vcm / NSV) & 1, abort_flag, P.status)) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.k_full[ks], (kcm / NSK) & 1, abort_flag, P.status))) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.v_full[vs], (vcm / NSV) & 1, abort_flag, P.status))) return false;
         }
         // buffer h is free once its epilogue is done and the dQ MMA read its dS
-        if (use > 0 && !mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
-        if (use > 0 && !mbar_wait(&sm.ds_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
+        if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status))) return false;
+        if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.ds_empty[h], (use - 1) & 1, abort_flag, P.status))) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(sm.k[ks]) + h * (kHalf * 128);
         const uint32_t v_addr = smem_u32(sm.v[vs]) + h * (kHalf * 128);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-          mma_f16_ss(tmem + 128 * h, smem_desc_sw128(q_addr + off, 16, 1024),
+          mma_f16_ss_warp(tmem + 128 * h, smem_desc_sw128(q_addr + off, 16, 1024),
                      smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-          mma_f16_ss(tmem + 128 * h + kHalf, smem_desc_sw128(do_addr + off, 16, 1024),
+          mma_f16_ss_warp(tmem + 128 * h + kHalf, smem_desc_sw128(do_addr + off, 16, 1024),
                      smem_desc_sw128(v_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sm.s_full[h]);
+        mma_commit_warp(&sm.s_full[h]);
         if (h == 0) ks_of0 = ks;
         else ks_of1 = ks;
         if (h == 1) {
-          mma_commit(&sm.v_empty[vs]);
+          mma_commit_warp(&sm.v_empty[vs]);
           ++kcm;
           ++vcm;
         }
@@ -340,19 +342,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // dQ += dS_h K_h for dQ step `dstep`
       auto issue_dq = [&]() -> bool {
         const uint32_t h = dstep & 1, use = dstep >> 1;
-        if (!mbar_wait(&sm.ds_full[h], use & 1, abort_flag, P.status)) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.ds_full[h], use & 1, abort_flag, P.status))) return false;
         tc_fence_after();
         const uint32_t ks = h == 0 ? ks_of0 : ks_of1;
         const uint32_t k_addr = smem_u32(sm.k[ks]) + h * (kHalf * 128);
 #pragma unroll
         for (int kk = 0; kk < kHalf / 16; ++kk) {
           const uint32_t a_col = 128 * h + (kk >> 1) * 32 + (kk & 1) * 8;
-          mma_f16_ts(tmem + kColDQ, tmem + a_col,
+          mma_f16_ts_warp(tmem + kColDQ, tmem + a_col,
                      smem_desc_sw128(k_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescDQ,
                      (dstep > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&sm.ds_empty[h]);
-        if (h == 1) mma_commit(&sm.k_empty[ks]);
+        mma_commit_warp(&sm.ds_empty[h]);
+        if (h == 1) mma_commit_warp(&sm.k_empty[ks]);
         ++dstep;
         return true;
       };
@@ -361,7 +363,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (u < 2 * n) ok = issue_sdp();
         if (ok && u > 0) ok = issue_dq();
       }
-      if (ok) mma_commit(&sm.dq_full);
+      if (ok) mma_commit_warp(&sm.dq_full);
       kc = kcm;
       vc = vcm;
     }
@@ -508,8 +510,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (uint32_t s = 0; s < NSV; ++s)
         if (vc > s) mbar_wait(&sm.v_full[s], ((vc - 1 - s) / NSV) & 1, nullptr, nullptr);
     }
-    if (warp == 1 && lane == 0) {
-      mma_commit(&sm.drain);
+    if (warp == 1) {
+      mma_commit_warp(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, nullptr);
     }
   }
@@ -654,33 +656,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(&sm.kv_full, 0, abort_flag, P.status);
+    // every lane runs the issue loop (warp-uniform descriptors); one elected
+    // lane issues each MMA and commit
+    {
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.kv_full, 0, abort_flag, P.status));
       const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
       // step u = 2 t + h: half h (query rows 64 h .. 64 h + 63) of active query tile t
       auto issue_s = [&](uint32_t u) -> bool {
         const uint32_t t = u >> 1, h = u & 1, slot = t % NS, use = u >> 1;
-        if (h == 0 && !mbar_wait(&sm.q_full[slot], (t / NS) & 1, abort_flag, P.status)) return false;
+        if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.q_full[slot], (t / NS) & 1, abort_flag, P.status))) return false;
         // buffer h is free once its epilogue is done and dV / dK read P^T / dS^T
-        if (use > 0 && !mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
-        if (use > 0 && !mbar_wait(&sm.pt_empty[h], (use - 1) & 1, abort_flag, P.status)) return false;
+        if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status))) return false;
+        if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.pt_empty[h], (use - 1) & 1, abort_flag, P.status))) return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm.q[slot]) + h * (kHalf * 128);
         const uint32_t do_addr = smem_u32(sm.dout[slot]) + h * (kHalf * 128);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-          mma_f16_ss(tmem + 128 * h, smem_desc_sw128(k_addr + off, 16, 1024),
+          mma_f16_ss_warp(tmem + 128 * h, smem_desc_sw128(k_addr + off, 16, 1024),
                      smem_desc_sw128(q_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-          mma_f16_ss(tmem + 128 * h + kHalf, smem_desc_sw128(v_addr + off, 16, 1024),
+          mma_f16_ss_warp(tmem + 128 * h + kHalf, smem_desc_sw128(v_addr + off, 16, 1024),
                      smem_desc_sw128(do_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sm.s_full[h]);
+        mma_commit_warp(&sm.s_full[h]);
         return true;
       };
       auto issue_acc = [&](uint32_t u) -> bool {
         const uint32_t t = u >> 1, h = u & 1, slot = t % NS, use = u >> 1;
-        if (!mbar_wait(&sm.pt_full[h], use & 1, abort_flag, P.status)) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.pt_full[h], use & 1, abort_flag, P.status))) return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm.q[slot]) + h * (kHalf * 128);
         const uint32_t do_addr = smem_u32(sm.dout[slot]) + h * (kHalf * 128);
@@ -688,14 +692,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int kk = 0; kk < kHalf / 16; ++kk) {
           const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
           const uint32_t a_col = 128 * h + (kk >> 1) * 32 + (kk & 1) * 8;
-          mma_f16_ts(tmem + kColDV, tmem + a_col,
+          mma_f16_ts_warp(tmem + kColDV, tmem + a_col,
                      smem_desc_sw128(do_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescAcc, acc);
           const uint64_t qd = smem_desc_sw128(q_addr + kk * 16 * 128, kSlabBytes, 1024);
-          mma_f16_ts(tmem + kColDK, tmem + a_col + kHalf, qd, kIdescAcc, acc);        // hi
-          mma_f16_ts(tmem + kColDK, tmem + a_col + kHalf + 16, qd, kIdescAcc, 1u);   // lo
+          mma_f16_ts_warp(tmem + kColDK, tmem + a_col + kHalf, qd, kIdescAcc, acc);        // hi
+          mma_f16_ts_warp(tmem + kColDK, tmem + a_col + kHalf + 16, qd, kIdescAcc, 1u);   // lo
         }
-        mma_commit(&sm.pt_empty[h]);
-        if (h == 1) mma_commit(&sm.q_empty[slot]);
+        mma_commit_warp(&sm.pt_empty[h]);
+        if (h == 1) mma_commit_warp(&sm.q_empty[slot]);
         return true;
       };
       const uint32_t steps = 2u * static_cast<uint32_t>(n);
@@ -707,7 +711,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (ok && u < steps) ok = issue_s(u);
         if (ok && !acc_first && u > 0) ok = issue_acc(u - 1);
       }
-      if (ok) mma_commit(&sm.acc_full);
+      if (ok) mma_commit_warp(&sm.acc_full);
     }
     __syncwarp();
   } else {
@@ -846,8 +850,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (uint32_t s = 0; s < NS; ++s)
         if (qc > s) mbar_wait(&sm.q_full[s], ((qc - 1 - s) / NS) & 1, nullptr, nullptr);
     }
-    if (warp == 1 && lane == 0) {
-      mma_commit(&sm.drain);
+    if (warp == 1) {
+      mma_commit_warp(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, nullptr);
     }
   }

@@ -180,13 +180,16 @@ __global__ void __launch_bounds__(kDashThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(&sm.kv_full, 0, abort_flag, P.status);
+    // every lane runs the issue loop (warp-uniform descriptors); one elected
+    // lane issues each MMA and commit
+    {
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.kv_full, 0, abort_flag, P.status));
       for (int g = 0; g < P.G && ok; ++g) {
         const int slot = g & 1;
-        ok = mbar_wait(&sm.q_full[slot], (g >> 1) & 1, abort_flag, P.status);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full[slot], (g >> 1) & 1, abort_flag, P.status));
         // the epilogue must be done with head g - 1's logits
-        if (ok && g > 0) ok = mbar_wait(&sm.s_free, (g - 1) & 1, abort_flag, P.status);
+        if (ok && g > 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_free, (g - 1) & 1, abort_flag, P.status));
         if (!ok) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm.q[slot]);
@@ -196,13 +199,13 @@ __global__ void __launch_bounds__(kDashThreads, 1)
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
             const uint64_t qd = smem_desc_sw128(q_addr + off, 16, 1024);
-            mma_f16_ss(tmem + ct * kTile, qd, smem_desc_sw128(hi_addr + off, 16, 1024), kIdesc,
+            mma_f16_ss_warp(tmem + ct * kTile, qd, smem_desc_sw128(hi_addr + off, 16, 1024), kIdesc,
                        kk > 0 ? 1u : 0u);
-            mma_f16_ss(tmem + ct * kTile, qd, smem_desc_sw128(lo_addr + off, 16, 1024), kIdesc, 1u);
+            mma_f16_ss_warp(tmem + ct * kTile, qd, smem_desc_sw128(lo_addr + off, 16, 1024), kIdesc, 1u);
           }
         }
-        mma_commit(&sm.s_full);
-        mma_commit(&sm.q_empty[slot]);
+        mma_commit_warp(&sm.s_full);
+        mma_commit_warp(&sm.q_empty[slot]);
       }
     }
     __syncwarp();
@@ -370,8 +373,8 @@ __global__ void __launch_bounds__(kDashThreads, 1)
       for (int s = 0; s < 2; ++s)
         if (qc > s) mbar_wait(&sm.q_full[s], ((qc - 1 - s) >> 1) & 1, nullptr, nullptr);
     }
-    if (warp == 1 && lane == 0) {
-      mma_commit(&sm.drain);
+    if (warp == 1) {
+      mma_commit_warp(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, nullptr);
     }
   }

@@ -592,29 +592,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       __syncwarp();
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
+      // every lane runs the issue loop (warp-uniform descriptors); one elected
+      // lane issues each MMA and commit
+      {
         bool ok = true;
         if (!q_waited) {
           q_waited = true;
-          ok = mbar_wait(&sm.q_full, 0, abort_flag, P.status);
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0, abort_flag, P.status));
         }
         const uint32_t q_addr = smem_u32(sm.q);
         auto issue_s = [&]() -> bool {
           const uint32_t slot = kc % NS;
-          if (!mbar_wait(&sm.k_full[slot], (kc / NS) & 1, abort_flag, P.status)) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.k_full[slot], (kc / NS) & 1, abort_flag, P.status))) return false;
           const uint32_t sb = sc % kNSB, use = sc / kNSB;
-          if (use > 0 && !mbar_wait(&sm.s_empty[sb], (use - 1) & 1, abort_flag, P.status))
+          if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.s_empty[sb], (use - 1) & 1, abort_flag, P.status)))
             return false;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(sm.k[slot]);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-            mma_f16_ss(tmem + sb * kTile, smem_desc_sw128(q_addr + off, 16, 1024),
+            mma_f16_ss_warp(tmem + sb * kTile, smem_desc_sw128(q_addr + off, 16, 1024),
                        smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
           }
-          mma_commit(&sm.s_full[sb]);
-          mma_commit(&sm.k_empty[slot]);
+          mma_commit_warp(&sm.s_full[sb]);
+          mma_commit_warp(&sm.k_empty[slot]);
           ++kc;
           ++sc;
           return true;
@@ -624,9 +626,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // columns 32 c .. 32 c + 31, P packed in the first 16, G in the last 16.
         auto issue_pv = [&](uint32_t sc0) -> bool {
           const uint32_t pb = pc % kNSB;
-          if (!mbar_wait(&sm.p_full[pb], (pc / kNSB) & 1, abort_flag, P.status)) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_full[pb], (pc / kNSB) & 1, abort_flag, P.status))) return false;
           const uint32_t slot = vc % NS;
-          if (!mbar_wait(&sm.v_full[slot], (vc / NS) & 1, abort_flag, P.status)) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.v_full[slot], (vc / NS) & 1, abort_flag, P.status))) return false;
           tc_fence_after();
           const uint32_t t_p = tmem + ((sc0 + pc) % kNSB) * kTile;
           const uint32_t v_addr = smem_u32(sm.v[slot]);
@@ -635,11 +637,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const uint32_t a_col = (kk >> 1) * 32 + (kk & 1) * 8;
             const uint64_t vd = smem_desc_sw128(v_addr + kk * 16 * 128, kSlabBytes, 1024);
             const uint32_t acc = (pc > 0 || kk > 0) ? 1u : 0u;
-            mma_f16_ts(tmem + kColO, t_p + a_col, vd, idesc_pv, acc);
-            if (gv) mma_f16_ts(tmem + kColG, t_p + a_col + 16, vd, idesc_pv, acc);
+            mma_f16_ts_warp(tmem + kColO, t_p + a_col, vd, idesc_pv, acc);
+            if (gv) mma_f16_ts_warp(tmem + kColG, t_p + a_col + 16, vd, idesc_pv, acc);
           }
-          mma_commit(&sm.v_empty[slot]);
-          mma_commit(&sm.p_empty[pb]);
+          mma_commit_warp(&sm.v_empty[slot]);
+          mma_commit_warp(&sm.p_empty[pb]);
           ++vc;
           ++pc;
           return true;
@@ -652,12 +654,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int t = 0; t <= n && ok; ++t) {
               // S(t) reuses the TMEM buffer of P.V tile t - kNSB: wait for its MMAs
               if (t < n && t >= static_cast<int>(kNSB))
-                ok = mbar_wait(&sm.p_empty[t % kNSB], ((t / kNSB) - 1) & 1, abort_flag,
-                               P.status);
+                ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_empty[t % kNSB], ((t / kNSB) - 1) & 1,
+                                                       abort_flag, P.status));
               if (ok && t < n) ok = issue_s();
               if (ok && t > 0) ok = issue_pv(sc0);
             }
-            if (ok) mma_commit(&sm.o_full);
+            if (ok) mma_commit_warp(&sm.o_full);
           }
         }
       }
@@ -1362,8 +1364,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (vc > s) mbar_wait(&sm.v_full[s], ((vc - 1 - s) / NS) & 1, nullptr, nullptr);
       }
     }
-    if (warp == 1 && lane == 0) {
-      mma_commit(&sm.drain);
+    if (warp == 1) {
+      mma_commit_warp(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, nullptr);
     }
   }

@@ -686,65 +686,79 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t t_s = t_lane + sb * kTile + hc0;
 
         if (kind == PASS_HIST) {
-          float tile_max = -INFINITY;
-          float cmx0 = -INFINITY, cmx1 = -INFINITY;
-#pragma unroll 1
-          for (int ch = 0; ch < 2; ++ch) {
-            uint32_t r[32];
-            tmem_ld32(t_s + ch * 32, r);
-            float v[32];
+          // Both 32-column chunks of this tile half are loaded under one wait,
+          // and the S buffer goes back to the MMA warp at once: the pass only
+          // reads the scores, and the candidate appends below use the registers.
+          uint32_t rr[2][32];
+          tmem_ld32x2(t_s, rr[0], t_s + 32, rr[1]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+          float v[2][32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
-            if (msk) apply_mask(v, j, ch);
-            // maxima of the four 8-score groups, then of the chunk (a tree)
-            float gm[4];
+          for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[ch][e] = __uint_as_float(rr[ch][e]);
+            if (msk) apply_mask(v[ch], j, ch);
+          }
+          // maxima of the 8-score groups and of each chunk (independent trees)
+          float gm[2][4], cmv[2];
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-              float a = fmaxf(fmaxf(v[8 * g], v[8 * g + 1]), fmaxf(v[8 * g + 2], v[8 * g + 3]));
-              float b = fmaxf(fmaxf(v[8 * g + 4], v[8 * g + 5]), fmaxf(v[8 * g + 6], v[8 * g + 7]));
-              gm[g] = fmaxf(a, b);
+              const float a = fmaxf(fmaxf(v[ch][8 * g], v[ch][8 * g + 1]),
+                                    fmaxf(v[ch][8 * g + 2], v[ch][8 * g + 3]));
+              const float b = fmaxf(fmaxf(v[ch][8 * g + 4], v[ch][8 * g + 5]),
+                                    fmaxf(v[ch][8 * g + 6], v[ch][8 * g + 7]));
+              gm[ch][g] = fmaxf(a, b);
             }
-            const float cm = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
-            tile_max = fmaxf(tile_max, cm);
-            m_raw = fmaxf(m_raw, cm);
-            if (cm > -INFINITY) {
-              const int gc = static_cast<int>(
-                  __float_as_uint(__fmaf_rd(fmaxf(cm, -P.slim), P.cN, kMagic)) - kMagicBits);
-              if (!gtop_set || gc > gtop) {
-                const int delta = gtop_set ? gc - gtop : kNB + 1;
-                if (delta > kNB) {
+            cmv[ch] = fmaxf(fmaxf(gm[ch][0], gm[ch][1]), fmaxf(gm[ch][2], gm[ch][3]));
+          }
+          const float tile_max = fmaxf(cmv[0], cmv[1]);
+          m_raw = fmaxf(m_raw, tile_max);
+          // one window update per tile half: binning both chunks against the
+          // window of the new running max leaves the same counts as binning
+          // chunk by chunk and shifting in between (the shift drops exactly the
+          // bins below the new window)
+          if (tile_max > -INFINITY) {
+            const int gc = static_cast<int>(
+                __float_as_uint(__fmaf_rd(fmaxf(tile_max, -P.slim), P.cN, kMagic)) - kMagicBits);
+            if (!gtop_set || gc > gtop) {
+              const int delta = gtop_set ? gc - gtop : kNB + 1;
+              if (delta > kNB) {
 #pragma unroll
-                  for (int b = 0; b <= kNB; ++b) cnt[b] = 0u;
-                } else {
-                  for (int d = 0; d < delta; ++d) {
+                for (int b = 0; b <= kNB; ++b) cnt[b] = 0u;
+              } else {
+                for (int d = 0; d < delta; ++d) {
 #pragma unroll
-                    for (int b = 0; b < kNB; ++b) cnt[b] = cnt[b + 1];
-                    cnt[kNB] = 0u;
-                  }
+                  for (int b = 0; b < kNB; ++b) cnt[b] = cnt[b + 1];
+                  cnt[kNB] = 0u;
                 }
-                gtop = gc;
-                gtop_set = true;
-                // Scores below the window are clamped to grid index <= base - 1,
-                // whose shift amount is "negative" and adds nothing.
-                vclamp = (static_cast<float>(gtop - kNB) - 1.5f) / P.cN;
-                cbase = 0u - 7u * (kMagicBits + static_cast<uint32_t>(gtop - kNB));
               }
+              gtop = gc;
+              gtop_set = true;
+              // Scores below the window are clamped to grid index <= base - 1,
+              // whose shift amount is "negative" and adds nothing.
+              vclamp = (static_cast<float>(gtop - kNB) - 1.5f) / P.cN;
+              cbase = 0u - 7u * (kMagicBits + static_cast<uint32_t>(gtop - kNB));
             }
-            // A chunk whose maximum lies below the window adds nothing to the
-            // histogram (common once the running max has settled): skip it.
-            // Only 8-score groups reaching the window add to the histogram (most
-            // scores of a long row lie far below it once the running max has
-            // settled).  9 bins in 7-bit lanes of 64-bit words: bin b of a score
-            // is floor(kNB * s) - (gtop - kNB), exact via a round-down FMA against
-            // 1.5 * 2^23; two independent words, lanes hold at most 32 counts.
-            if (cm > vclamp) {
+          }
+          // Only 8-score groups reaching the window add to the histogram (most
+          // scores of a long row lie far below it once the running max has
+          // settled).  9 bins in 7-bit lanes of 64-bit words: bin b of a score
+          // is floor(kNB * s) - (gtop - kNB), exact via a round-down FMA against
+          // 1.5 * 2^23; two independent words, lanes hold at most 32 counts.
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            if (cmv[ch] > vclamp) {
               uint64_t pk0 = 0, pk1 = 0;
 #pragma unroll
               for (int g = 0; g < 4; ++g) {
-                if (gm[g] > vclamp) {
+                if (gm[ch][g] > vclamp) {
 #pragma unroll
                   for (int e = 8 * g; e < 8 * g + 8; ++e) {
-                    const float u = __fmaf_rd(fmaxf(v[e], vclamp), P.cN, kMagic);
+                    const float u = __fmaf_rd(fmaxf(v[ch][e], vclamp), P.cN, kMagic);
                     const uint32_t sh = __float_as_uint(u) * 7u + cbase;
                     if (e & 1) pk1 += shl64(1ull, sh);
                     else pk0 += shl64(1ull, sh);
@@ -756,32 +770,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               for (int b = 0; b <= kNB; ++b)
                 cnt[b] += static_cast<uint32_t>(packed >> (7 * b)) & 127u;
             }
-            if (ch == 0) cmx0 = cm;
-            else cmx1 = cm;
           }
           // Candidates of this tile half: every score above acc_raw, raised to a
           // lower bound of the partial histogram's tau_h (scores seen so far by
           // this warpgroup, so <= tau*) whenever a chunk reaches the current bound.
           {
             acc_raw = fmaxf(acc_raw, __fsub_rd(m_raw, P.inv_c));
-            if (row_ok && !cand_over && gtop_set && fmaxf(cmx0, cmx1) > acc_raw) {
+            if (row_ok && !cand_over && gtop_set && tile_max > acc_raw) {
               const float lb = GEN ? hist_lower_bound_gen(cnt, gtop, P.kpow, P.am1)
                                    : hist_lower_bound<ALPHA2>(cnt, gtop);   // s-units
               acc_raw = fmaxf(acc_raw, lb * (lb >= 0.0f ? P.inv_c_dn : P.inv_c));
             }
           }
-#pragma unroll 1
-          for (int ch = 0; ch < 2; ++ch) {
-            const float cm = ch == 0 ? cmx0 : cmx1;
-            const bool want = row_ok && !cand_over && cm > acc_raw;
-            if (!__any_sync(0xffffffffu, want)) continue;
-            uint32_t r[32];
-            tmem_ld32(t_s + ch * 32, r);
-            if (!want) continue;
-            float v[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
-            if (msk) apply_mask(v, j, ch);
+          for (int ch = 0; ch < 2; ++ch) {
+            const bool want = row_ok && !cand_over && cmv[ch] > acc_raw;
+            if (!want) continue;
             if (ncand + 32 > kCapH) {
               if (prunes < kMaxPrunes) {
                 ++prunes;
@@ -797,13 +801,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!cand_over) {
 #pragma unroll
               for (int e = 0; e < 32; ++e) {
-                if (v[e] > acc_raw) cand_put(ncand++, v[e]);
+                if (v[ch][e] > acc_raw) cand_put(ncand++, v[ch][e]);
               }
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
           const float rec = row_ok ? tile_max * P.c : -INFINITY;
           const size_t ti = tmax_index(bh, i, j, P.tr, P.tc, P.causal) + wg * kTile + rl;
           if (in_bounds(ti < tmax_elems)) P.tmax[ti] = __float2half_ru(rec);

@@ -481,6 +481,70 @@ def run_ours(args, points, rank, world, device):
     return line
 
 
+def dense_context(args, points, results, device):
+    """Dense causal softmax attention, forward + backward, on the same shapes:
+    torch's scaled_dot_product_attention (whichever backend it dispatches to) and,
+    if it runs on this GPU, the flash_attn package (FlashAttention-2), each timed
+    like our step (CUDA events, L2 flushed before each step).  Context for the
+    pages' comparison with FlashAttention-2 at high block sparsity: a different
+    function (softmax, not entmax), never a parity or speed-up claim."""
+    import torch.nn.functional as F
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    out = []
+    for w, r in zip(points, results):
+        x = W.make_inputs(w, device="cpu")
+        q, k, v, do = (x[n].to(device) for n in ("q", "k", "v", "dout"))
+        entry = {"point": w.name, "block_sparsity": r["block_sparsity"],
+                 "entmax_ms_per_step": r["ms_per_step"]}
+
+        def timed(fn):
+            for _ in range(max(3, args.warmup)):
+                fn()
+            torch.cuda.synchronize(device)
+            ev0 = torch.cuda.Event(enable_timing=True)
+            ev1 = torch.cuda.Event(enable_timing=True)
+            tot = 0.0
+            for _ in range(args.steps):
+                flush.zero_()
+                ev0.record()
+                fn()
+                ev1.record()
+                ev1.synchronize()
+                tot += ev0.elapsed_time(ev1)
+            return round(tot / args.steps, 4)
+
+        qs, ks, vs = (t.detach().clone().requires_grad_(True) for t in (q, k, v))
+
+        def sdpa_step():
+            o = F.scaled_dot_product_attention(qs, ks, vs, is_causal=True)
+            o.backward(do)
+        try:
+            entry["sdpa_ms_per_step"] = timed(sdpa_step)
+        except Exception as e:  # noqa: BLE001 - context only
+            entry["sdpa_ms_per_step"] = None
+            entry["sdpa_error"] = str(e).splitlines()[0][:200]
+        del qs, ks, vs
+        try:
+            from flash_attn import flash_attn_func
+            qf, kf, vf = (t.transpose(1, 2).contiguous().requires_grad_(True) for t in (q, k, v))
+            dof = do.transpose(1, 2).contiguous()
+
+            def fa2_step():
+                o = flash_attn_func(qf, kf, vf, causal=True)
+                o.backward(dof)
+            entry["flash_attn2_ms_per_step"] = timed(fa2_step)
+            del qf, kf, vf, dof
+        except Exception as e:  # noqa: BLE001 - context only
+            entry["flash_attn2_ms_per_step"] = None
+            entry["flash_attn2_error"] = str(e).splitlines()[0][:200]
+        out.append(entry)
+        del q, k, v, do
+        torch.cuda.empty_cache()
+    return {"note": "dense causal softmax attention fwd+bwd on the same shapes (bf16): a "
+                    "different function, timed as context for the pages' comparison only",
+            "points": out}
+
+
 def merge_clocks(cl):
     sm = [c["sm_mhz"] for c in cl if c.get("sm_mhz")]
     reasons = sorted({r for c in cl for r in c.get("reasons", [])})
@@ -739,6 +803,9 @@ def main():
                     help="override alpha (any value in [1.05, 3]; 1.5 and 2 have closed forms)")
     ap.add_argument("--block", type=int, default=0, choices=[0, 64, 128],
                     help="override the mask block size (the sparsity is then reported at it)")
+    ap.add_argument("--dense-context", action="store_true",
+                    help="also time dense causal softmax attention (torch SDPA, flash_attn) "
+                         "on the same shapes, as context")
     args = ap.parse_args()
     if args.workload == "dash_router_16k":
         world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -790,6 +857,8 @@ def main():
                                              timeout=datetime.timedelta(seconds=120))
     line = run_ours(args, points, rank, world, device)
     if rank == 0:
+        if args.dense_context and world == 1:
+            line["dense_context"] = dense_context(args, points, line["sweep"], device)
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(points)
         print(json.dumps(line))

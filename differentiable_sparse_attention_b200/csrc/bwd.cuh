@@ -168,7 +168,8 @@ __device__ __forceinline__ int load_tile_list(const uint32_t* rowbits, int wt, u
 // buffering) and the MMAs of one half overlap the epilogue of the other.
 // Two epilogue warpgroups (warps 2-5 and 6-9) alternate: warpgroup h owns half
 // h of every tile and its TMEM / SMEM buffer.
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 352;   // warp 0 TMA, warps 1 and 10 MMA, warps 2-9 epilogue
+constexpr int kAccWarp = 10;       // issues the accumulating MMAs (dQ; dV and dK)
 constexpr int kHalf = 64;
 constexpr int kHalfBytes = kTile * kHalf * 2;   // one [128][64] fp16 slab
 
@@ -188,7 +189,7 @@ struct BwdRowSmem {
   uint64_t qdo_full;
   uint64_t k_full[NSK], k_empty[NSK];
   uint64_t v_full[NSV], v_empty[NSV];
-  uint64_t s_full[2], s_empty[2], ds_full[2], ds_empty[2], dq_full, drain;
+  uint64_t s_full[2], s_empty[2], ds_full[2], ds_empty[2], dq_full, drain, drain_acc;
   uint32_t tmem_base;
   int abort_flag;
   int ntiles;
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain_acc, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -297,26 +299,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    // every lane runs the issue loop (warp-uniform descriptors); one elected
-    // lane issues each MMA and commit
+    // ---------------------------------------------------------------- S / dP issuer
+    // Two warps issue the MMAs: this one S and dP, warp kAccWarp the dQ steps.
+    // A wait in one warp then leaves the other's MMAs running on the tensor
+    // pipe.  Every lane runs the issue loop (warp-uniform descriptors); one
+    // elected lane issues each MMA and commit.
     {
       bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.qdo_full, 0, abort_flag, P.status));
       const uint32_t q_addr = smem_u32(sm.q), do_addr = smem_u32(sm.dout);
-      uint32_t step = 0, dstep = 0;     // half-tile steps issued (S/dP) and dQ steps issued
       uint32_t kcm = 0, vcm = 0;        // K / V tiles consumed
-      uint32_t ks_of0 = 0, ks_of1 = 0;  // K slot of the tile each buffer's step belongs to
-      // S = Q K_h^T and dP = dO V_h^T of step `step` (half h of the current tile)
-      auto issue_sdp = [&]() -> bool {
-        const uint32_t h = step & 1, use = step >> 1;
+      // S = Q K_h^T and dP = dO V_h^T of step u (half h of tile u / 2)
+      for (uint32_t u = 0; u < 2u * static_cast<uint32_t>(n) && ok; ++u) {
+        const uint32_t h = u & 1, use = u >> 1;
         const uint32_t ks = kcm % NSK, vs = vcm % NSV;
         if (h == 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.k_full[ks], (kcm / NSK) & 1, abort_flag, P.status))) return false;
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.v_full[vs], (vcm / NSV) & 1, abort_flag, P.status))) return false;
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.k_full[ks], (kcm / NSK) & 1, abort_flag, P.status));
+          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.v_full[vs], (vcm / NSV) & 1, abort_flag, P.status));
+          if (!ok) break;
         }
-        // buffer h is free once its epilogue is done and the dQ MMA read its dS
-        if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status))) return false;
-        if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.ds_empty[h], (use - 1) & 1, abort_flag, P.status))) return false;
+        // buffer h is free once its epilogue is done and the dQ MMAs read its dS
+        if (use > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status));
+          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.ds_empty[h], (use - 1) & 1, abort_flag, P.status));
+          if (!ok) break;
+        }
         tc_fence_after();
         const uint32_t k_addr = smem_u32(sm.k[ks]) + h * (kHalf * 128);
         const uint32_t v_addr = smem_u32(sm.v[vs]) + h * (kHalf * 128);
@@ -329,43 +335,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                      smem_desc_sw128(v_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
         mma_commit_warp(&sm.s_full[h]);
-        if (h == 0) ks_of0 = ks;
-        else ks_of1 = ks;
         if (h == 1) {
           mma_commit_warp(&sm.v_empty[vs]);
           ++kcm;
           ++vcm;
         }
-        ++step;
-        return true;
-      };
-      // dQ += dS_h K_h for dQ step `dstep`
-      auto issue_dq = [&]() -> bool {
-        const uint32_t h = dstep & 1, use = dstep >> 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.ds_full[h], use & 1, abort_flag, P.status))) return false;
+      }
+    }
+    __syncwarp();
+  } else if (warp == kAccWarp) {
+    // ---------------------------------------------------------------- dQ issuer
+    // dQ += dS_h K_h for step u, once the epilogue has written dS_h (ds_full).
+    // K of tile t sits in slot t % NSK: the S issuer consumed it in that order,
+    // and it stays until this warp's k_empty commit after the tile's second half.
+    {
+      bool ok = true;
+      for (uint32_t u = 0; u < 2u * static_cast<uint32_t>(n) && ok; ++u) {
+        const uint32_t h = u & 1, use = u >> 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.ds_full[h], use & 1, abort_flag, P.status));
+        if (!ok) break;
         tc_fence_after();
-        const uint32_t ks = h == 0 ? ks_of0 : ks_of1;
+        const uint32_t ks = use % NSK;
         const uint32_t k_addr = smem_u32(sm.k[ks]) + h * (kHalf * 128);
 #pragma unroll
         for (int kk = 0; kk < kHalf / 16; ++kk) {
           const uint32_t a_col = 128 * h + (kk >> 1) * 32 + (kk & 1) * 8;
           mma_f16_ts_warp(tmem + kColDQ, tmem + a_col,
                      smem_desc_sw128(k_addr + kk * 16 * 128, kSlabBytes, 1024), kIdescDQ,
-                     (dstep > 0 || kk > 0) ? 1u : 0u);
+                     (u > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit_warp(&sm.ds_empty[h]);
         if (h == 1) mma_commit_warp(&sm.k_empty[ks]);
-        ++dstep;
-        return true;
-      };
-      // dQ steps trail the S/dP steps by one
-      for (int u = 0; u <= 2 * n && ok; ++u) {
-        if (u < 2 * n) ok = issue_sdp();
-        if (ok && u > 0) ok = issue_dq();
       }
       if (ok) mma_commit_warp(&sm.dq_full);
-      kc = kcm;
-      vc = vcm;
     }
     __syncwarp();
   } else {
@@ -514,6 +516,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit_warp(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, nullptr);
     }
+    if (warp == kAccWarp) {
+      mma_commit_warp(&sm.drain_acc);
+      mbar_wait(&sm.drain_acc, 0, nullptr, nullptr);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -532,7 +538,7 @@ struct BwdColSmem {
   float delta[NS][kTile];
   uint64_t kv_full;
   uint64_t q_full[NS], q_empty[NS];
-  uint64_t s_full[2], s_empty[2], pt_full[2], pt_empty[2], acc_full, drain;
+  uint64_t s_full[2], s_empty[2], pt_full[2], pt_empty[2], acc_full, drain, drain_acc;
   uint32_t tmem_base;
   int abort_flag;
   int ntiles;
@@ -592,6 +598,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain_acc, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -655,19 +662,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    // every lane runs the issue loop (warp-uniform descriptors); one elected
-    // lane issues each MMA and commit
+    // ---------------------------------------------------------------- S^T / dP^T issuer
+    // Two warps issue the MMAs: this one S^T and dP^T, warp kAccWarp the dV / dK
+    // accumulation.  A wait in one warp then leaves the other's MMAs running on
+    // the tensor pipe.  Every lane runs the issue loop (warp-uniform
+    // descriptors); one elected lane issues each MMA and commit.
     {
       bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.kv_full, 0, abort_flag, P.status));
       const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
       // step u = 2 t + h: half h (query rows 64 h .. 64 h + 63) of active query tile t
-      auto issue_s = [&](uint32_t u) -> bool {
+      for (uint32_t u = 0; u < 2u * static_cast<uint32_t>(n) && ok; ++u) {
         const uint32_t t = u >> 1, h = u & 1, slot = t % NS, use = u >> 1;
-        if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.q_full[slot], (t / NS) & 1, abort_flag, P.status))) return false;
+        if (h == 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full[slot], (t / NS) & 1, abort_flag, P.status));
+          if (!ok) break;
+        }
         // buffer h is free once its epilogue is done and dV / dK read P^T / dS^T
-        if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status))) return false;
-        if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.pt_empty[h], (use - 1) & 1, abort_flag, P.status))) return false;
+        if (use > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status));
+          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.pt_empty[h], (use - 1) & 1, abort_flag, P.status));
+          if (!ok) break;
+        }
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm.q[slot]) + h * (kHalf * 128);
         const uint32_t do_addr = smem_u32(sm.dout[slot]) + h * (kHalf * 128);
@@ -680,11 +695,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                      smem_desc_sw128(do_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
         mma_commit_warp(&sm.s_full[h]);
-        return true;
-      };
-      auto issue_acc = [&](uint32_t u) -> bool {
+      }
+    }
+    __syncwarp();
+  } else if (warp == kAccWarp) {
+    // ---------------------------------------------------------------- dV / dK issuer
+    // dV += P^T_h dO_h and dK += dS^T_h Q_h (dS^T as two fp16 parts) for step u,
+    // once the epilogue has written P^T and dS^T (pt_full); the Q / dO slot of
+    // tile t is released after its second half.
+    {
+      bool ok = true;
+      for (uint32_t u = 0; u < 2u * static_cast<uint32_t>(n) && ok; ++u) {
         const uint32_t t = u >> 1, h = u & 1, slot = t % NS, use = u >> 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.pt_full[h], use & 1, abort_flag, P.status))) return false;
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.pt_full[h], use & 1, abort_flag, P.status));
+        if (!ok) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm.q[slot]) + h * (kHalf * 128);
         const uint32_t do_addr = smem_u32(sm.dout[slot]) + h * (kHalf * 128);
@@ -700,16 +724,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mma_commit_warp(&sm.pt_empty[h]);
         if (h == 1) mma_commit_warp(&sm.q_empty[slot]);
-        return true;
-      };
-      const uint32_t steps = 2u * static_cast<uint32_t>(n);
-      for (uint32_t u = 0; u <= steps && ok; ++u) {
-        // With one Q / dO stage the previous tile's last accumulation must free
-        // it before the next tile's first S^T step can be loaded.
-        const bool acc_first = NS == 1 && (u & 1) == 0;
-        if (acc_first && u > 0) ok = issue_acc(u - 1);
-        if (ok && u < steps) ok = issue_s(u);
-        if (ok && !acc_first && u > 0) ok = issue_acc(u - 1);
       }
       if (ok) mma_commit_warp(&sm.acc_full);
     }
@@ -853,6 +867,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (warp == 1) {
       mma_commit_warp(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, nullptr);
+    }
+    if (warp == kAccWarp) {
+      mma_commit_warp(&sm.drain_acc);
+      mbar_wait(&sm.drain_acc, 0, nullptr, nullptr);
     }
   }
   tc_fence_before();

@@ -288,7 +288,9 @@ __device__ __forceinline__ bool solver_step(double F0, double F1, double F2, flo
   return exact;
 }
 
-constexpr int kFwdThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int kFwdThreads = 352;   // warp 0 TMA, warp 1 S MMAs, warps 2-9 epilogue, warp 10 P.V MMAs
+constexpr int kFwdEpiThreads = 256;
+constexpr int kPvWarp = 10;
 
 __device__ __forceinline__ void fwd_epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 // The same barrier, returning whether v held for any of the 256 threads.
@@ -332,7 +334,7 @@ struct FwdSmem {
   // S buffers in TMEM: three at D = 64 (3 x 128 + 2 x 64 columns), two at 128
   static constexpr int kNSB = D == 64 ? 3 : 2;
   uint64_t s_full[kNSB], s_empty[kNSB];
-  uint64_t p_full[kNSB], p_empty[kNSB], o_full, drain;
+  uint64_t p_full[kNSB], p_empty[kNSB], o_full, drain, drain_pv;
   uint32_t tmem_base;
   int abort_flag;
   int ctl_kind, ctl_n, ctl_iter;
@@ -446,6 +448,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain_pv, 1);
     sm.abort_flag = 0;
     sm.not_converged = 0;
     sm.cand_overflow = 0;
@@ -591,9 +594,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       __syncwarp();
     } else if (warp == 1) {
-      // ------------------------------------------------------------ MMA issuer
-      // every lane runs the issue loop (warp-uniform descriptors); one elected
-      // lane issues each MMA and commit
+      // ------------------------------------------------------------ S issuer
+      // S = Q K^T of every pass.  In the P.V pass warp kPvWarp issues the P.V
+      // MMAs, so a wait in one warp leaves the other's MMAs running on the
+      // tensor pipe.  Every lane runs the issue loop (warp-uniform
+      // descriptors); one elected lane issues each MMA and commit.
       {
         bool ok = true;
         if (!q_waited) {
@@ -601,12 +606,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0, abort_flag, P.status));
         }
         const uint32_t q_addr = smem_u32(sm.q);
-        auto issue_s = [&]() -> bool {
+        for (int t = 0; t < n && ok; ++t) {
           const uint32_t slot = kc % NS;
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.k_full[slot], (kc / NS) & 1, abort_flag, P.status))) return false;
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.k_full[slot], (kc / NS) & 1, abort_flag, P.status));
+          if (!ok) break;
           const uint32_t sb = sc % kNSB, use = sc / kNSB;
-          if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.s_empty[sb], (use - 1) & 1, abort_flag, P.status)))
-            return false;
+          if (use > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_empty[sb], (use - 1) & 1, abort_flag, P.status));
+            if (!ok) break;
+          }
+          // In the P.V pass S(t) reuses the TMEM buffer of P.V tile t - kNSB:
+          // wait for those MMAs too
+          if (kind == PASS_PV && t >= static_cast<int>(kNSB)) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_empty[t % kNSB], ((t / kNSB) - 1) & 1,
+                                                   abort_flag, P.status));
+            if (!ok) break;
+          }
           tc_fence_after();
           const uint32_t k_addr = smem_u32(sm.k[slot]);
 #pragma unroll
@@ -619,16 +634,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mma_commit_warp(&sm.k_empty[slot]);
           ++kc;
           ++sc;
-          return true;
-        };
-        // O += P V and (with the g-weighted means) G.V += G V for P.V tile pc.
-        // P and G sit in the S buffer of their tile: 32-key chunk c occupies
-        // columns 32 c .. 32 c + 31, P packed in the first 16, G in the last 16.
-        auto issue_pv = [&](uint32_t sc0) -> bool {
+        }
+      }
+      __syncwarp();
+    } else if (warp == kPvWarp) {
+      // ------------------------------------------------------------ P.V issuer
+      // O += P V and (with the g-weighted means) G.V += G V for P.V tile t.
+      // P and G sit in the S buffer of their tile: 32-key chunk c occupies
+      // columns 32 c .. 32 c + 31, P packed in the first 16, G in the last 16.
+      // sc follows the S issuer's count (n S tiles per pass) so that tile t's
+      // buffer is (S count at the pass start + t) % kNSB.
+      if (kind == PASS_PV) {
+        bool ok = true;
+        const uint32_t sc0 = sc;
+        for (int t = 0; t < n && ok; ++t) {
           const uint32_t pb = pc % kNSB;
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_full[pb], (pc / kNSB) & 1, abort_flag, P.status))) return false;
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[pb], (pc / kNSB) & 1, abort_flag, P.status));
+          if (!ok) break;
           const uint32_t slot = vc % NS;
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.v_full[slot], (vc / NS) & 1, abort_flag, P.status))) return false;
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.v_full[slot], (vc / NS) & 1, abort_flag, P.status));
+          if (!ok) break;
           tc_fence_after();
           const uint32_t t_p = tmem + ((sc0 + pc) % kNSB) * kTile;
           const uint32_t v_addr = smem_u32(sm.v[slot]);
@@ -644,25 +669,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mma_commit_warp(&sm.p_empty[pb]);
           ++vc;
           ++pc;
-          return true;
-        };
-        if (ok) {
-          if (kind != PASS_PV) {
-            for (int t = 0; t < n && ok; ++t) ok = issue_s();
-          } else {
-            const uint32_t sc0 = sc;
-            for (int t = 0; t <= n && ok; ++t) {
-              // S(t) reuses the TMEM buffer of P.V tile t - kNSB: wait for its MMAs
-              if (t < n && t >= static_cast<int>(kNSB))
-                ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_empty[t % kNSB], ((t / kNSB) - 1) & 1,
-                                                       abort_flag, P.status));
-              if (ok && t < n) ok = issue_s();
-              if (ok && t > 0) ok = issue_pv(sc0);
-            }
-            if (ok) mma_commit_warp(&sm.o_full);
-          }
         }
+        if (ok) mma_commit_warp(&sm.o_full);
       }
+      sc += static_cast<uint32_t>(n);
       __syncwarp();
     } else {
       // ------------------------------------------------------------ epilogue
@@ -1337,7 +1347,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int it = iter + 1; it <= P.max_iter; ++it) trace_store(it, tau_c);
         const int spr = kTile / P.block;
         const int et = threadIdx.x - 64;
-        for (int idx = et; idx < spr * P.mask_words; idx += kFwdThreads - 64) {
+        for (int idx = et; idx < spr * P.mask_words; idx += kFwdEpiThreads) {
           const int h = idx / P.mask_words;
           const int w = idx - h * P.mask_words;
           const int mrow = i * spr + h;
@@ -1368,6 +1378,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (warp == 1) {
       mma_commit_warp(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, nullptr);
+    }
+    if (warp == kPvWarp) {
+      mma_commit_warp(&sm.drain_pv);
+      mbar_wait(&sm.drain_pv, 0, nullptr, nullptr);
     }
   }
   tc_fence_before();

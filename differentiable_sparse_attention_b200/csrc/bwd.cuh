@@ -168,8 +168,9 @@ __device__ __forceinline__ int load_tile_list(const uint32_t* rowbits, int wt, u
 // buffering) and the MMAs of one half overlap the epilogue of the other.
 // Two epilogue warpgroups (warps 2-5 and 6-9) alternate: warpgroup h owns half
 // h of every tile and its TMEM / SMEM buffer.
-constexpr int kBwdThreads = 352;   // warp 0 TMA, warps 1 and 10 MMA, warps 2-9 epilogue
+constexpr int kBwdThreads = 384;   // warp 0 TMA, warps 1, 10 and 11 MMA, warps 2-9 epilogue
 constexpr int kAccWarp = 10;       // issues the accumulating MMAs (dQ; dV and dK)
+constexpr int kDpWarp = 11;        // issues dP (dP^T); warp 1 issues S (S^T)
 constexpr int kHalf = 64;
 constexpr int kHalfBytes = kTile * kHalf * 2;   // one [128][64] fp16 slab
 
@@ -189,7 +190,7 @@ struct BwdRowSmem {
   uint64_t qdo_full;
   uint64_t k_full[NSK], k_empty[NSK];
   uint64_t v_full[NSV], v_empty[NSV];
-  uint64_t s_full[2], s_empty[2], ds_full[2], ds_empty[2], dq_full, drain, drain_acc;
+  uint64_t s_full[2], s_empty[2], ds_full[2], ds_empty[2], dq_full, drain, drain_acc, drain_dp;
   uint32_t tmem_base;
   int abort_flag;
   int ntiles;
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int s = 0; s < NSK; ++s) { mbar_init(&sm.k_full[s], 1); mbar_init(&sm.k_empty[s], 1); }
     for (int s = 0; s < NSV; ++s) { mbar_init(&sm.v_full[s], 1); mbar_init(&sm.v_empty[s], 1); }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_full[b], 2);   // the S and the dP issuer each commit once
       mbar_init(&sm.s_empty[b], 4);
       mbar_init(&sm.ds_full[b], 4);
       mbar_init(&sm.ds_empty[b], 1);
@@ -244,6 +245,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.drain_acc, 1);
+    mbar_init(&sm.drain_dp, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -298,47 +300,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- S / dP issuer
-    // Two warps issue the MMAs: this one S and dP, warp kAccWarp the dQ steps.
-    // A wait in one warp then leaves the other's MMAs running on the tensor
-    // pipe.  Every lane runs the issue loop (warp-uniform descriptors); one
+  } else if (warp == 1 || warp == kDpWarp) {
+    // ---------------------------------------------------------------- S and dP issuers
+    // Three warps issue the MMAs: warp 1 S = Q K_h^T, warp kDpWarp dP = dO V_h^T,
+    // warp kAccWarp the dQ steps.  A wait in one warp then leaves the others'
+    // MMAs running on the tensor pipe, and each waits only for its own operand
+    // (K or V).  Every lane runs the issue loop (warp-uniform descriptors); one
     // elected lane issues each MMA and commit.
     {
+      const bool is_s = warp == 1;
       bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.qdo_full, 0, abort_flag, P.status));
-      const uint32_t q_addr = smem_u32(sm.q), do_addr = smem_u32(sm.dout);
-      uint32_t kcm = 0, vcm = 0;        // K / V tiles consumed
-      // S = Q K_h^T and dP = dO V_h^T of step u (half h of tile u / 2)
+      const uint32_t a_addr = is_s ? smem_u32(sm.q) : smem_u32(sm.dout);
+      const uint32_t d_col = is_s ? 0u : static_cast<uint32_t>(kHalf);
+      uint32_t tcn = 0;   // tiles consumed
+      // step u is half h of tile u / 2
       for (uint32_t u = 0; u < 2u * static_cast<uint32_t>(n) && ok; ++u) {
         const uint32_t h = u & 1, use = u >> 1;
-        const uint32_t ks = kcm % NSK, vs = vcm % NSV;
+        const uint32_t ks = tcn % NSK, vs = tcn % NSV;
         if (h == 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&sm.k_full[ks], (kcm / NSK) & 1, abort_flag, P.status));
-          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.v_full[vs], (vcm / NSV) & 1, abort_flag, P.status));
+          ok = is_s ? __all_sync(0xffffffffu, mbar_wait(&sm.k_full[ks], (tcn / NSK) & 1, abort_flag, P.status))
+                    : __all_sync(0xffffffffu, mbar_wait(&sm.v_full[vs], (tcn / NSV) & 1, abort_flag, P.status));
           if (!ok) break;
         }
-        // buffer h is free once its epilogue is done and the dQ MMAs read its dS
+        // buffer h is free once its epilogue is done; the S columns also hold the
+        // dS that the dQ MMAs of step u - 2 read
         if (use > 0) {
           ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_empty[h], (use - 1) & 1, abort_flag, P.status));
-          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.ds_empty[h], (use - 1) & 1, abort_flag, P.status));
+          if (ok && is_s) ok = __all_sync(0xffffffffu, mbar_wait(&sm.ds_empty[h], (use - 1) & 1, abort_flag, P.status));
           if (!ok) break;
         }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm.k[ks]) + h * (kHalf * 128);
-        const uint32_t v_addr = smem_u32(sm.v[vs]) + h * (kHalf * 128);
+        const uint32_t b_addr = (is_s ? smem_u32(sm.k[ks]) : smem_u32(sm.v[vs])) + h * (kHalf * 128);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-          mma_f16_ss_warp(tmem + 128 * h, smem_desc_sw128(q_addr + off, 16, 1024),
-                     smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-          mma_f16_ss_warp(tmem + 128 * h + kHalf, smem_desc_sw128(do_addr + off, 16, 1024),
-                     smem_desc_sw128(v_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          mma_f16_ss_warp(tmem + 128 * h + d_col, smem_desc_sw128(a_addr + off, 16, 1024),
+                     smem_desc_sw128(b_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
         mma_commit_warp(&sm.s_full[h]);
         if (h == 1) {
-          mma_commit_warp(&sm.v_empty[vs]);
-          ++kcm;
-          ++vcm;
+          if (!is_s) mma_commit_warp(&sm.v_empty[vs]);
+          ++tcn;
         }
       }
     }
@@ -520,6 +522,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit_warp(&sm.drain_acc);
       mbar_wait(&sm.drain_acc, 0, nullptr, nullptr);
     }
+    if (warp == kDpWarp) {
+      mma_commit_warp(&sm.drain_dp);
+      mbar_wait(&sm.drain_dp, 0, nullptr, nullptr);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -538,7 +544,7 @@ struct BwdColSmem {
   float delta[NS][kTile];
   uint64_t kv_full;
   uint64_t q_full[NS], q_empty[NS];
-  uint64_t s_full[2], s_empty[2], pt_full[2], pt_empty[2], acc_full, drain, drain_acc;
+  uint64_t s_full[2], s_empty[2], pt_full[2], pt_empty[2], acc_full, drain, drain_acc, drain_dp;
   uint32_t tmem_base;
   int abort_flag;
   int ntiles;
@@ -591,7 +597,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&sm.q_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_full[b], 2);   // the S^T and the dP^T issuer each commit once
       mbar_init(&sm.s_empty[b], 4);
       mbar_init(&sm.pt_full[b], 4);
       mbar_init(&sm.pt_empty[b], 1);
@@ -599,6 +605,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.drain_acc, 1);
+    mbar_init(&sm.drain_dp, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -661,15 +668,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ++qc;
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- S^T / dP^T issuer
-    // Two warps issue the MMAs: this one S^T and dP^T, warp kAccWarp the dV / dK
-    // accumulation.  A wait in one warp then leaves the other's MMAs running on
-    // the tensor pipe.  Every lane runs the issue loop (warp-uniform
-    // descriptors); one elected lane issues each MMA and commit.
+  } else if (warp == 1 || warp == kDpWarp) {
+    // ---------------------------------------------------------------- S^T and dP^T issuers
+    // Three warps issue the MMAs: warp 1 S^T = K Q_h^T, warp kDpWarp
+    // dP^T = V dO_h^T, warp kAccWarp the dV / dK accumulation.  A wait in one
+    // warp then leaves the others' MMAs running on the tensor pipe.  Every lane
+    // runs the issue loop (warp-uniform descriptors); one elected lane issues
+    // each MMA and commit.
     {
+      const bool is_s = warp == 1;
       bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.kv_full, 0, abort_flag, P.status));
-      const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+      const uint32_t a_addr = is_s ? smem_u32(sm.k) : smem_u32(sm.v);
+      const uint32_t d_col = is_s ? 0u : static_cast<uint32_t>(kHalf);
       // step u = 2 t + h: half h (query rows 64 h .. 64 h + 63) of active query tile t
       for (uint32_t u = 0; u < 2u * static_cast<uint32_t>(n) && ok; ++u) {
         const uint32_t t = u >> 1, h = u & 1, slot = t % NS, use = u >> 1;
@@ -684,15 +694,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!ok) break;
         }
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sm.q[slot]) + h * (kHalf * 128);
-        const uint32_t do_addr = smem_u32(sm.dout[slot]) + h * (kHalf * 128);
+        const uint32_t b_addr = (is_s ? smem_u32(sm.q[slot]) : smem_u32(sm.dout[slot])) + h * (kHalf * 128);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-          mma_f16_ss_warp(tmem + 128 * h, smem_desc_sw128(k_addr + off, 16, 1024),
-                     smem_desc_sw128(q_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-          mma_f16_ss_warp(tmem + 128 * h + kHalf, smem_desc_sw128(v_addr + off, 16, 1024),
-                     smem_desc_sw128(do_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          mma_f16_ss_warp(tmem + 128 * h + d_col, smem_desc_sw128(a_addr + off, 16, 1024),
+                     smem_desc_sw128(b_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
         mma_commit_warp(&sm.s_full[h]);
       }
@@ -871,6 +878,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (warp == kAccWarp) {
       mma_commit_warp(&sm.drain_acc);
       mbar_wait(&sm.drain_acc, 0, nullptr, nullptr);
+    }
+    if (warp == kDpWarp) {
+      mma_commit_warp(&sm.drain_dp);
+      mbar_wait(&sm.drain_dp, 0, nullptr, nullptr);
     }
   }
   tc_fence_before();

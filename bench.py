@@ -44,8 +44,17 @@ from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
 # DRAM bytes (read + write) per launch of a kernel from one ncu capture, keyed
 # by (sweep point, kernel) and valid only for the kernel code they were taken
 # on (hash of the package's csrc/ with comments and white space removed); any
-# other code reports traffic as null.
-TRAFFIC = {}
+# other code reports traffic as null.  Each figure is dram__bytes_read.sum +
+# dram__bytes_write.sum of the timed step's forward launch of that point's own
+# workload at full size (a one-pass capture, after the L2 flush).
+_TRAFFIC_SRC = "45488c640e22285c"
+TRAFFIC = {
+    ("long_n65536_alpha1.5_t4", "fwd"): {"bytes": 969773824 + 929166848, "src": _TRAFFIC_SRC},
+    ("long_n131072_alpha1.5_t4", "fwd"): {"bytes": 3045766144 + 2992464384, "src": _TRAFFIC_SRC},
+    ("long_n65536_alpha2.0_t4", "fwd"): {"bytes": 917882112 + 926514688, "src": _TRAFFIC_SRC},
+    ("long_n131072_alpha2.0_t4", "fwd"): {"bytes": 3094034432 + 2981843712, "src": _TRAFFIC_SRC},
+    ("alpha1.5_n4096_d64", "fwd"): {"bytes": 51154944 + 16886016, "src": _TRAFFIC_SRC},
+}
 
 
 def _code_only(text: str) -> str:

@@ -697,7 +697,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
         if (kind == PASS_HIST) {
           // Both 32-column chunks of this tile half are loaded under one wait,
-          // and the S buffer goes back to the MMA warp at once: the pass only
+          // and the S buffer goes back to the S issuer at once: the pass only
           // reads the scores, and the candidate appends below use the registers.
           uint32_t rr[2][32];
           tmem_ld32x2(t_s, rr[0], t_s + 32, rr[1]);
@@ -890,8 +890,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           Tmin = fminf(Tmin, fminf(fminf(tmin[0], tmin[1]), fminf(tmin[2], tmin[3])));
           Tneg = fmaxf(Tneg, fmaxf(fmaxf(tneg[0], tneg[1]), fmaxf(tneg[2], tneg[3])));
         } else {  // PASS_PV
-          // P (and G) replace the scores in this S buffer; the MMA warp issues
-          // S(t + 2) into it only after the P.V MMAs of this tile completed.
+          // P (and G) replace the scores in this S buffer; the S issuer puts
+          // S(t + kNSB) into it only after the P.V MMAs of this tile completed.
           const uint32_t pb = pc % kNSB;
           ++pc;
           float part = 0.f, gpart = 0.f;

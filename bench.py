@@ -47,13 +47,13 @@ from differentiable_sparse_attention_b200 import workloads as W  # noqa: E402
 # other code reports traffic as null.  Each figure is dram__bytes_read.sum +
 # dram__bytes_write.sum of the timed step's forward launch of that point's own
 # workload at full size (a one-pass capture, after the L2 flush).
-_TRAFFIC_SRC = "45488c640e22285c"
+_TRAFFIC_SRC = "52624589d9a02622"
 TRAFFIC = {
-    ("long_n65536_alpha1.5_t4", "fwd"): {"bytes": 969773824 + 929166848, "src": _TRAFFIC_SRC},
-    ("long_n131072_alpha1.5_t4", "fwd"): {"bytes": 3045766144 + 2992464384, "src": _TRAFFIC_SRC},
-    ("long_n65536_alpha2.0_t4", "fwd"): {"bytes": 917882112 + 926514688, "src": _TRAFFIC_SRC},
-    ("long_n131072_alpha2.0_t4", "fwd"): {"bytes": 3094034432 + 2981843712, "src": _TRAFFIC_SRC},
-    ("alpha1.5_n4096_d64", "fwd"): {"bytes": 51154944 + 16886016, "src": _TRAFFIC_SRC},
+    ("long_n65536_alpha1.5_t4", "fwd"): {"bytes": 971897088 + 932220672, "src": _TRAFFIC_SRC},
+    ("long_n131072_alpha1.5_t4", "fwd"): {"bytes": 3933710592 + 3003946752, "src": _TRAFFIC_SRC},
+    ("long_n65536_alpha2.0_t4", "fwd"): {"bytes": 917617664 + 927312896, "src": _TRAFFIC_SRC},
+    ("long_n131072_alpha2.0_t4", "fwd"): {"bytes": 3161120768 + 2982609664, "src": _TRAFFIC_SRC},
+    ("alpha1.5_n4096_d64", "fwd"): {"bytes": 51134720 + 16934912, "src": _TRAFFIC_SRC},
 }
 
 
